@@ -1,0 +1,348 @@
+"""Pins for the CPU oracle: format facts, brute force, closed forms and invariants.
+
+Nothing here re-types the oracle's formulas: every expectation comes from the
+format definition (golden file), an exhaustive search, an exact special case or
+a mathematical identity, chosen so that a dropped term, a wrong sign, a wrong
+index or a transposed operand in the oracle fails at least one test.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import layout
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_format_facts.json")
+
+
+@pytest.fixture(scope="module")
+def facts():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ------------------------------------------------------------------ E2M1 pins
+def test_e2m1_decode_matches_value_set(facts):
+    vals = oracle.e2m1_decode(np.arange(16))
+    want = np.array(facts["e2m1_values_by_code"])
+    assert np.array_equal(vals, want)
+    assert np.array_equal(np.signbit(vals), np.signbit(want))
+
+
+def _brute_e2m1(v):
+    """Nearest of the 8 magnitudes by exhaustive search; ties to the even code."""
+    mags = [abs(x) for x in json.load(open(GOLDEN))["e2m1_values_by_code"][:8]]
+    best = None
+    for code, m in enumerate(mags):
+        d = abs(abs(v) - m)
+        if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
+            best = (d, code)
+    code = best[1]
+    if math.copysign(1.0, v) < 0:
+        code |= 8
+    return code
+
+
+def test_e2m1_encode_brute_force_sweep():
+    # dense sweep over [-8, 8] including every midpoint and every representable value
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    grid = np.unique(np.concatenate([np.linspace(-8, 8, 4097), mids, -mids,
+                                     [6.0, 7.0, 1e6, -1e6, 0.2499999, 0.2500001]]))
+    got = oracle.e2m1_encode(grid)
+    want = np.array([_brute_e2m1(float(v)) for v in grid], dtype=np.uint8)
+    assert np.array_equal(got, want)
+
+
+def test_e2m1_threshold_table(facts):
+    rules = facts["e2m1_round_to_nearest_even_thresholds"]["rules"]
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.uniform(0, 8, 20000),
+                        np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])])
+    got = np.abs(oracle.e2m1_decode(oracle.e2m1_encode(v)))
+    for x, g in zip(v, got):
+        for op, t, mag in rules:
+            if op == "else" or (op == "<=" and x <= t) or (op == "<" and x < t):
+                assert g == mag, (x, g, mag)
+                break
+
+
+def test_e2m1_sign_of_zero():
+    assert oracle.e2m1_encode(np.array([-0.0]))[0] == 0x8
+    assert oracle.e2m1_encode(np.array([-0.1]))[0] == 0x8
+    assert oracle.e2m1_encode(np.array([0.1]))[0] == 0x0
+    assert oracle.e2m1_encode(np.array([-0.3]))[0] == 0x9
+
+
+# ------------------------------------------------------------------ E4M3 pins
+def test_e4m3_known_values(facts):
+    for hexs, val in facts["e4m3_known"]:
+        d = oracle.e4m3_decode(int(hexs, 16))
+        assert d == val and np.signbit(d) == np.signbit(val), hexs
+    for hexs in facts["e4m3_nan"]:
+        assert np.isnan(oracle.e4m3_decode(int(hexs, 16)))
+    pos = oracle.e4m3_decode(np.arange(1, 128))
+    assert np.sum(np.isfinite(pos) & (pos > 0)) == facts["e4m3_finite_positive_count"]
+    # strictly increasing with the code over the finite non-negative range
+    fin = oracle.e4m3_decode(np.arange(0x7F))
+    assert np.all(np.diff(fin) > 0)
+
+
+_E4M3_TABLE = [float(oracle.e4m3_decode(c)) for c in range(0x7F)]
+
+
+def _brute_e4m3(s):
+    best = None
+    for code, val in enumerate(_E4M3_TABLE):
+        d = abs(s - val)
+        if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
+            best = (d, code)
+    return best[1]
+
+
+def test_e4m3_encode_brute_force():
+    rng = np.random.default_rng(5)
+    fin = oracle.e4m3_decode(np.arange(0x7F))
+    mids = (fin[1:] + fin[:-1]) / 2
+    s = np.concatenate([rng.uniform(0, 500, 3000), np.exp(rng.uniform(-14, 6.5, 3000)),
+                        mids, fin, [448.0, 449.0, 464.0, 480.0, 1e9, 0.0, 2.0 ** -10, 2.0 ** -11]])
+    s = s.astype(np.float32).astype(np.float64)
+    got = oracle.e4m3_encode(s)
+    want = np.array([_brute_e4m3(float(x)) for x in s], dtype=np.uint8)
+    assert np.array_equal(got, want)
+    assert oracle.e4m3_encode(np.array([1e30]))[0] == 0x7E
+
+
+# ---------------------------------------------------------------- quantiser pins
+def _random_block_matrix(rng, rows, cols, spread=True):
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    if spread:
+        x *= np.exp(rng.uniform(-6, 6, (rows, cols // 16, 1))).repeat(16, axis=2).reshape(rows, cols).astype(np.float32)
+    return synth.bf16_to_f32(synth.f32_to_bf16_bits(x))
+
+
+def test_global_scale_definition():
+    x = np.array([[0.5, -2688.0] + [0.0] * 14], dtype=np.float32)
+    assert oracle.global_scale(x) == np.float32(1.0)
+    assert oracle.global_scale(np.zeros((2, 16), np.float32)) == np.float32(1.0)
+    x = np.array([[3.0] * 16], dtype=np.float32)
+    assert oracle.global_scale(x) == np.float32(896.0)
+
+
+def test_roundtrip_of_representable_blocks():
+    """A block of E2M1 values times 2**e containing +-6*2**e quantises back to itself (gs = 1)."""
+    rng = np.random.default_rng(11)
+    vals = oracle.e2m1_decode(np.arange(16))
+    rows, cols = 64, 64
+    codes = rng.integers(0, 16, (rows, cols)).astype(np.uint8)
+    codes[:, ::16] = np.where(rng.random((rows, cols // 16)) < 0.5, 7, 15)  # each block has +-6
+    e = rng.integers(-5, 7, (rows, cols // 16))
+    x = (vals[codes] * np.ldexp(1.0, e).repeat(16, axis=1)).astype(np.float32)
+    qc, sf = oracle.quantize(x, np.float32(1.0))
+    # +0 / -0 both decode to 0: compare values and signs of non-zero codes
+    assert np.array_equal(oracle.e2m1_decode(qc), vals[codes])
+    assert np.array_equal(qc[vals[codes] != 0], codes[vals[codes] != 0])
+    assert np.array_equal(oracle.e4m3_decode(sf), np.ldexp(1.0, e))
+
+
+def test_block_amax_maps_to_six_and_largest_block_to_448():
+    rng = np.random.default_rng(12)
+    x = _random_block_matrix(rng, 48, 256)
+    gs = oracle.global_scale(x)
+    codes, sf = oracle.quantize(x, gs)
+    xb = np.abs(x.reshape(48, 16, 16))
+    arg = xb.argmax(axis=2)
+    cb = codes.reshape(48, 16, 16)
+    top = np.take_along_axis(cb, arg[:, :, None], axis=2)[:, :, 0]
+    normal = sf >= 0x08
+    assert np.all((top[normal] & 7) == 7)
+    # the block holding the tensor amax gets the largest scale, 448
+    r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert sf[r, c // 16] == 0x7E
+    assert sf.max() == 0x7E
+
+
+def test_zero_block():
+    x = np.zeros((2, 32), np.float32)
+    x[1, 16:] = -0.0
+    x[0, 16:] = np.linspace(-1, 1, 16)
+    codes, sf = oracle.quantize(x, np.float32(3.0))
+    assert sf[0, 0] == 0 and sf[1, 0] == 0 and sf[1, 1] == 0
+    assert np.all(codes[0, :16] == 0)
+    assert np.all(codes[1, 16:] == 8)  # -0 keeps its sign bit (reading R2)
+
+
+def test_quantize_elementwise_optimal_given_scale():
+    """Brute force: sf is the nearest E4M3 of s, and every code is the nearest of all 16 codes to x*gs/dec(sf)."""
+    rng = np.random.default_rng(13)
+    x = _random_block_matrix(rng, 6, 64)
+    gs = oracle.global_scale(x)
+    codes, sf = oracle.quantize(x, gs)
+    allv = oracle.e2m1_decode(np.arange(16))
+    for r in range(6):
+        for j in range(4):
+            blk = x[r, 16 * j:16 * j + 16]
+            amax = np.float32(np.max(np.abs(blk)))
+            s = np.float32(np.float32(amax / np.float32(6)) * gs)
+            assert sf[r, j] == _brute_e4m3(float(s))
+            dec = float(oracle.e4m3_decode(sf[r, j]))
+            inv = np.float32(0) if dec == 0 else np.float32(gs / np.float32(dec))
+            for i in range(16):
+                v = float(np.float32(blk[i] * inv))
+                d = np.abs(allv - v)
+                best = d.min()
+                cand = [c for c in range(16) if d[c] == best]
+                assert codes[r, 16 * j + i] in cand
+                c = int(codes[r, 16 * j + i])
+                if len({c & 7 for c in cand}) > 1:   # tie: even mantissa wins
+                    assert c % 2 == 0
+
+
+def test_dequant_error_sanity_band():
+    """Not a pin: relative round-trip error on outlier activations lands near the blog's 7.5-9.2 %."""
+    x = synth.bf16_to_f32(synth.outlier_activations(64, 1024, seed=0))
+    gs = oracle.global_scale(x)
+    codes, sf = oracle.quantize(x, gs)
+    xh = oracle.dequantize(codes, sf, gs)
+    rel = np.linalg.norm(xh - x) / np.linalg.norm(x)
+    assert 0.03 < rel < 0.2
+
+
+# ------------------------------------------------------------------ GEMM pins
+def test_linear_textbook_triple_loop():
+    rng = np.random.default_rng(21)
+    M, N, K = 3, 5, 32
+    a = _random_block_matrix(rng, M, K)
+    w = _random_block_matrix(rng, N, K)
+    gs_a = oracle.global_scale(a)
+    ca, sa = oracle.quantize(a, gs_a)
+    gsw = [np.float32(7.0), np.float32(0.25)]
+    cw, sw = oracle.quantize(w, np.float32(1.0))
+    segs = [(0, 2, gsw[0]), (2, 5, gsw[1])]
+    y = oracle.linear(ca, sa, gs_a, cw, sw, segs)
+    vals = json.load(open(GOLDEN))["e2m1_values_by_code"]
+    e4 = dict((int(h, 16), v) for h, v in json.load(open(GOLDEN))["e4m3_known"])
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += (vals[ca[m, k]] * float(oracle.e4m3_decode(sa[m, k // 16]))
+                        * vals[cw[n, k]] * float(oracle.e4m3_decode(sw[n, k // 16])))
+            g = gsw[0] if n < 2 else gsw[1]
+            assert math.isclose(y[m, n], acc / (float(gs_a) * float(g)), rel_tol=1e-12, abs_tol=1e-300)
+    assert e4[0x38] == 1.0
+
+
+def test_linear_exact_small_integer_case():
+    """gs = 1 and every scale = 1.0 (0x38): 2*Y is an integer matrix product."""
+    rng = np.random.default_rng(22)
+    M, N, K = 17, 9, 128
+    ca = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    cw = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sa = np.full((M, K // 16), 0x38, np.uint8)
+    sw = np.full((N, K // 16), 0x38, np.uint8)
+    twice = np.array([0, 1, 2, 3, 4, 6, 8, 12, 0, -1, -2, -3, -4, -6, -8, -12], dtype=np.int64)
+    want = (twice[ca] @ twice[cw].T) / 4.0
+    y = oracle.linear(ca, sa, np.float32(1), cw, sw, [(0, N, np.float32(1))])
+    assert np.array_equal(y, want)
+
+
+def test_fused_equals_separate_modules():
+    """One GEMM over concatenated segments with per-segment alpha == the per-module GEMMs."""
+    rng = np.random.default_rng(23)
+    K = 64
+    x = _random_block_matrix(rng, 10, K)
+    gs_a = oracle.global_scale(x)
+    ca, sa = oracle.quantize(x, gs_a)
+    mods = [(_random_block_matrix(rng, 16, K) * s).astype(np.float32) for s in (1, 8, 16)]
+    sep, codes, scales, segs, n0 = [], [], [], [], 0
+    for w in mods:
+        gw = oracle.global_scale(w)
+        cw, sw = oracle.quantize(w, gw)
+        sep.append(oracle.linear(ca, sa, gs_a, cw, sw, [(0, 16, gw)]))
+        codes.append(cw), scales.append(sw), segs.append((n0, n0 + 16, gw))
+        n0 += 16
+    fused = oracle.linear(ca, sa, gs_a, np.concatenate(codes), np.concatenate(scales), segs)
+    assert np.array_equal(fused, np.concatenate(sep, axis=1))
+    # one shared scale (the mismatch the pages describe) is measurably wrong
+    wrong = oracle.linear(ca, sa, gs_a, np.concatenate(codes), np.concatenate(scales),
+                          [(0, 48, segs[0][2])])
+    assert not np.allclose(wrong, fused, rtol=1e-2)
+
+
+# ---------------------------------------------------------------- epilogue pins
+def test_gate_closed_forms(facts):
+    cf = facts["gate_closed_forms"]
+    assert oracle.sigmoid(0.0) == cf["sigmoid_at_0"]
+    assert math.isclose(oracle.softplus(0.0), cf["softplus_at_0"], rel_tol=1e-15)
+    a_log = np.array([0.3, -1.2])
+    dt = np.array([0.5, -0.25])
+    beta, g = oracle.gdn_gates(np.zeros((1, 2)), -dt[None, :], a_log, dt)
+    assert np.allclose(beta, 0.5)
+    assert np.allclose(g, -np.exp(a_log) * cf["softplus_at_0"], rtol=1e-15)
+    x = np.linspace(-30, 30, 601)
+    assert np.allclose(oracle.sigmoid(x) + oracle.sigmoid(-x), 1.0, atol=1e-15)
+    assert np.allclose(oracle.softplus(x) - oracle.softplus(-x), x, atol=1e-12)
+    assert np.allclose(oracle.silu(x) - oracle.silu(-x), x, atol=1e-12)
+    assert np.all(np.diff(oracle.softplus(x)) > 0) and np.all(oracle.softplus(x) > 0)
+    # decay gate is negative and decreasing in a
+    _, g = oracle.gdn_gates(np.zeros((601, 1)), x[:, None], np.array([0.0]), np.array([0.0]))
+    assert np.all(g < 0) and np.all(np.diff(g[:, 0]) < 0)
+    assert np.allclose(oracle.silu_mul(np.array([0.0, 2.0]), np.array([5.0, 3.0])),
+                       [0.0, 6.0 / (1.0 + math.exp(-2.0))])
+
+
+def test_round_to_bf16_agrees_with_independent_rounders():
+    import torch
+    rng = np.random.default_rng(31)
+    x32 = (rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))).astype(np.float32)
+    ours = oracle.round_to_bf16(x32.astype(np.float64))
+    via_synth = synth.bf16_to_f32(synth.f32_to_bf16_bits(x32)).astype(np.float64)
+    via_torch = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(ours, via_synth)
+    assert np.array_equal(ours, via_torch)
+    # exact ties in FP64 go to even
+    assert oracle.round_to_bf16(1.0 + 2.0 ** -8) == 1.0
+    assert oracle.round_to_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+
+
+# ------------------------------------------------------------------- layout
+def test_scale_layout_reading():
+    cols = 512  # 32 blocks -> 8 atoms per 128-row group
+    assert layout.scale_offset(0, 0, cols) == 0
+    assert layout.scale_offset(0, 1, cols) == 1
+    assert layout.scale_offset(1, 0, cols) == 16
+    assert layout.scale_offset(32, 0, cols) == 4
+    assert layout.scale_offset(96, 3, cols) == 15
+    assert layout.scale_offset(0, 4, cols) == 512
+    assert layout.scale_offset(128, 0, cols) == 8 * 512
+    rng = np.random.default_rng(41)
+    for rows, c in [(1, 16), (130, 80), (300, 512)]:
+        sf = rng.integers(0, 255, (rows, c // 16)).astype(np.uint8)
+        buf = layout.swizzle_scales(sf, rows, c)
+        assert buf.size == layout.scale_bytes(rows, c)
+        assert np.array_equal(layout.unswizzle_scales(buf, rows, c), sf)
+        # offsets are a bijection onto the non-padding bytes
+        r, j = np.meshgrid(np.arange(rows), np.arange(c // 16), indexing="ij")
+        offs = layout.scale_offset(r, j, c).ravel()
+        assert len(np.unique(offs)) == offs.size
+
+
+def test_nibble_packing_reading():
+    codes = np.array([[1, 2, 3, 4, 15, 0]], np.uint8)
+    p = layout.pack_nibbles(codes)
+    assert p.tolist() == [[0x21, 0x43, 0x0F]]
+    assert np.array_equal(layout.unpack_nibbles(p), codes)
+
+
+def test_synth_is_seeded_and_bf16():
+    a = synth.outlier_activations(8, 64, seed=0)
+    b = synth.outlier_activations(8, 64, seed=0)
+    assert a.dtype == np.uint16 and np.array_equal(a, b)
+    t = synth.student_t_activations(16, 128, seed=0)
+    x = synth.bf16_to_f32(t)
+    assert np.all(np.isfinite(x))
