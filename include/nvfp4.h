@@ -1,0 +1,199 @@
+/*
+ * nvfp4.h - C ABI of the B200 (sm_100a) NVFP4 W4A4 linear library.
+ *
+ * The method: every linear layer of a hybrid Gated-DeltaNet / attention LLM runs
+ * with both weights and activations in NVFP4 (W4A4): 4-bit E2M1 values, one E4M3
+ * scale per 16 consecutive elements, and one FP32 global scale per tensor; the
+ * GEMM runs on 4-bit tensor cores.  Sources: blog "27BハイブリッドLLMを4ビットで動かす
+ * ——Gated DeltaNetはなぜ量子化に耐えるのか", sections 機構① (block format, block maximum
+ * sets the scale), 機構② (GDN gate formulas), 罠① (per-module global scales in a
+ * fused GEMM) and FAQ; abstract page "Why Gated DeltaNet Survives 4-Bit
+ * Quantization" (arXiv 2609.04098).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *   allocates, frees or keeps them; it launches work on `stream` and returns
+ *   without synchronising.  Results are valid once the stream reaches that point.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  The current
+ *   CUDA device must be the device that owns the pointers.
+ * - Matrices are row-major.  BF16 inputs are IEEE bfloat16 bit patterns.
+ * - Packed NVFP4 codes: two E2M1 codes per byte, the element with the even column
+ *   index in the low nibble; row r of a [rows x cols] tensor starts at byte r*cols/2.
+ * - Block scales: unsigned E4M3 bytes, one per 16-element row block, stored in
+ *   512-byte atoms of 128 rows x 4 blocks: row r, block j of an atom sits at byte
+ *   (r%32)*16 + (r/32)*4 + j; atoms are ordered block-index fastest; rows are
+ *   padded to a multiple of 128 and blocks to a multiple of 4 (padding written as 0
+ *   by nvfp4_quantize).  This is the layout the tcgen05 block-scaled MMA reads.
+ * - Global scale: gs = 2688 / amax(|x|) (2688 = 448 * 6), FP32, in device memory;
+ *   a quantised value means e2m1(code) * e4m3(scale) / gs.
+ * - Errors are returned, never printed, and no kernel is launched when a check fails.
+ *   NVFP4_ERR_CUDA means a CUDA runtime call failed (cudaGetLastError is left set).
+ */
+#ifndef NVFP4_W4A4_H
+#define NVFP4_W4A4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nvfp4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, unknown enum value */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size violates the documented divisibility rules */
+  NVFP4_ERR_MISALIGNED = 3,        /* a pointer or leading dimension violates alignment */
+  NVFP4_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
+  NVFP4_ERR_DEVICE_TIMEOUT = 5,    /* a kernel gave up a bounded wait (see nvfp4_get_device_status) */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 6 /* current device is not sm_100 */
+} nvfp4_status_t;
+
+/* Human-readable name of a status code (static storage). */
+NVFP4_API const char *nvfp4_status_string(int status);
+
+/* Bytes of the swizzled scale buffer of a [rows x cols] NVFP4 tensor:
+ * ceil(rows/128)*128 * ceil(cols/64)*4.  Returns 0 for invalid sizes. */
+NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t cols);
+
+/*
+ * nvfp4_global_scale - per-tensor FP32 global scale from the tensor's amax.
+ *   Computes gs = fl32(2688 / max|x|) over x [rows x cols] (row stride `ld`
+ *   elements) and writes it to *gs_out (device).  max|x| == 0 gives gs = 1.
+ *   Source: blog section 罠① (each linear module has its own global scale); the
+ *   formula is this library's reading (the pages give none).
+ *   Requirements: rows, cols >= 1; ld >= cols; x 16-byte aligned and ld % 8 == 0;
+ *   gs_out 4-byte aligned.  Non-finite inputs are unsupported.
+ */
+NVFP4_API nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                  float *gs_out, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_quantize - NVFP4 block quantisation of a BF16 matrix.
+ *   For each 16-element row block b of x [rows x cols]:
+ *     s    = fl32(fl32(amax_b / 6) * gs)
+ *     sf_b = E4M3(s)  (round to nearest even, saturate at 448)
+ *     code = E2M1(fl32(x * fl32(gs / e4m3(sf_b))))  (nearest even, saturate at 6,
+ *            sign copied; 0 when sf_b == 0)
+ *   Source: blog section 機構① (16-element blocks, E4M3 block scale set by the block
+ *   maximum, E2M1 values).  Operation order and rounding are this library's reading.
+ *   x: device BF16, row stride ld elements (ld >= cols, ld % 8 == 0, 16-byte aligned).
+ *   gs: device FP32 scalar (static calibrated scale, or nvfp4_global_scale's output).
+ *   codes: device, rows*cols/2 bytes, 16-byte aligned.
+ *   scales: device, nvfp4_scale_bytes(rows, cols) bytes, 16-byte aligned; padding
+ *   bytes are written with 0.
+ *   Requirements: rows >= 1, cols >= 16, cols % 16 == 0.
+ */
+NVFP4_API nvfp4_status_t nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                              const float *gs, uint8_t *codes, uint8_t *scales,
+                              nvfp4_stream_t stream);
+
+/*
+ * nvfp4_quantize_rows - nvfp4_quantize into rows [row_offset, row_offset + rows) of
+ *   a larger destination tensor of total_rows rows (same cols): `codes` and
+ *   `scales` are the buffers of the whole destination.  This packs a fused weight
+ *   whose modules keep their own global scales (blog section 罠①): one call per
+ *   module, each with its own gs, into one weight.  Scale bytes of other rows are
+ *   untouched, except that the call that ends at total_rows also zero-fills the
+ *   padding rows up to a multiple of 128.  Calls on disjoint row ranges may run
+ *   concurrently.  nvfp4_quantize(...) == nvfp4_quantize_rows(..., 0, rows, ...).
+ *   Requirements as nvfp4_quantize, plus 0 <= row_offset, row_offset + rows <= total_rows.
+ */
+NVFP4_API nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                             const float *gs, uint8_t *codes, uint8_t *scales,
+                                             int64_t row_offset, int64_t total_rows, nvfp4_stream_t stream);
+
+/* A quantised operand of the GEMM: [rows x K] NVFP4, both K-major. */
+typedef struct {
+  const uint8_t *codes;  /* device, rows*K/2 bytes, 16-byte aligned */
+  const uint8_t *scales; /* device, nvfp4_scale_bytes(rows, K) bytes, 16-byte aligned */
+  int64_t rows;
+  int64_t K;
+} nvfp4_operand_t;
+
+/* One separately calibrated module inside a fused weight: weight rows (= output
+ * columns of the GEMM) [n_begin, n_end) carry global scale *gs_w (device). */
+typedef struct {
+  int64_t n_begin;
+  int64_t n_end;
+  const float *gs_w;
+} nvfp4_segment_t;
+
+#define NVFP4_MAX_SEGMENTS 16
+
+typedef enum {
+  NVFP4_EPI_NONE = 0,      /* y = alpha(n) * acc */
+  NVFP4_EPI_SILU_MUL = 1,  /* W = [gate; up] (2*Nh rows): y[:, j] = SiLU(y_gate[:, j]) * y_up[:, j] */
+  NVFP4_EPI_GDN_GATES = 2  /* columns of the beta head block -> sigmoid; of the alpha block -> g */
+} nvfp4_epilogue_t;
+
+typedef enum {
+  NVFP4_OUT_BF16 = 0,  /* out: BF16 [M x Nout], row stride ldo elements */
+  NVFP4_OUT_F32 = 1,   /* out: FP32 [M x Nout], row stride ldo elements */
+  NVFP4_OUT_NVFP4 = 2  /* out: packed codes [M x Nout/2] (ldo ignored) + ep->out_scales,
+                          quantised with ep->gs_out after rounding y to BF16 */
+} nvfp4_out_kind_t;
+
+typedef struct {
+  /* NVFP4_EPI_GDN_GATES: g = -exp(A_log[h]) * softplus(y + dt_bias[h]) on columns
+   * [alpha_begin, alpha_begin + n_heads), beta = sigmoid(y) on columns
+   * [beta_begin, beta_begin + n_heads); h = column - block begin.  The gated values
+   * replace y in `out`; when non-NULL, FP32 copies go to beta_out / g_out
+   * ([M x n_heads], row stride n_heads). */
+  int64_t beta_begin;
+  int64_t alpha_begin;
+  int64_t n_heads;
+  const float *A_log;   /* device [n_heads] */
+  const float *dt_bias; /* device [n_heads] */
+  float *beta_out;      /* device or NULL */
+  float *g_out;         /* device or NULL */
+  /* NVFP4_OUT_NVFP4: global scale of the output (device scalar) and its scale buffer
+   * (nvfp4_scale_bytes(M, Nout) bytes). */
+  const float *gs_out;
+  uint8_t *out_scales;
+} nvfp4_epilogue_params_t;
+
+/*
+ * nvfp4_linear - fused W4A4 linear: block-scaled FP4 x FP4 GEMM on tcgen05 tensor
+ * cores with per-segment global-scale correction and a selectable epilogue.
+ *   acc[m, n] = sum_k e2m1(A)[m,k] e4m3(sfA)[m,k/16] e2m1(W)[n,k] e4m3(sfW)[n,k/16]  (FP32)
+ *   y[m, n]   = acc[m, n] / (gs_a * gs_w(seg(n)))
+ *   then the epilogue; out = epilogue(y) stored as `out_kind`.
+ *   Sources: blog FAQ (W4A4 on 4-bit tensor cores), section 罠① (fused modules need
+ *   their own global-scale correction; here a per-segment alpha), section 機構② (gates).
+ *   A: [M x K] activations; gs_a: device FP32 scalar.  W: [N x K] weights.
+ *   segs/nseg: 1..16 segments, sorted, disjoint, covering [0, N); bounds % 16 == 0.
+ *   Requirements: M >= 1; K % 256 == 0; N % 16 == 0; for SILU_MUL, N % 256 == 0
+ *   and Nout = N/2, else Nout = N; ldo >= Nout; out 16-byte aligned and ldo*elem % 16 == 0;
+ *   NVFP4 output needs Nout % 64 == 0.  GDN_GATES needs n_heads >= 1 and both head
+ *   blocks inside [0, N).
+ *   ep may be NULL for NVFP4_EPI_NONE with BF16/F32 output.
+ */
+NVFP4_API nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
+                            const nvfp4_segment_t *segs, int nseg, int epilogue,
+                            const nvfp4_epilogue_params_t *ep, void *out, int out_kind,
+                            int64_t ldo, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_get_device_status - read and clear the device status word of the current
+ * device.  Kernels never spin forever: every wait on an mbarrier has an iteration
+ * limit, and a wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the
+ * kernel returns.  *code receives NVFP4_OK (0) when nothing was recorded.
+ * Synchronises the device.
+ */
+NVFP4_API nvfp4_status_t nvfp4_get_device_status(int *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_W4A4_H */

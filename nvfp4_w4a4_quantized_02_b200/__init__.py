@@ -1,0 +1,233 @@
+"""Python binding of the B200 NVFP4 W4A4 linear library (``include/nvfp4.h``).
+
+Argument marshalling only: every step of the quantiser and of the linear runs in
+the CUDA kernels of ``libnvfp4_w4a4.so``.  PyTorch supplies device memory (the
+caller-side output buffers allocated here) and the current CUDA stream.  There is
+no CPU fallback: if the library is missing or the device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+__all__ = [
+    "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
+    "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4_w4a4.so")
+
+EPILOGUES = {"none": 0, "silu_mul": 1, "gdn_gates": 2}
+OUT_KINDS = {"bf16": 0, "f32": 1, "nvfp4": 2}
+MAX_SEGMENTS = 16
+
+_c_i64 = ctypes.c_int64
+_c_vp = ctypes.c_void_p
+
+
+class Operand(ctypes.Structure):
+    _fields_ = [("codes", _c_vp), ("scales", _c_vp), ("rows", _c_i64), ("K", _c_i64)]
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("n_begin", _c_i64), ("n_end", _c_i64), ("gs_w", _c_vp)]
+
+
+class EpilogueParams(ctypes.Structure):
+    _fields_ = [("beta_begin", _c_i64), ("alpha_begin", _c_i64), ("n_heads", _c_i64),
+                ("A_log", _c_vp), ("dt_bias", _c_vp), ("beta_out", _c_vp), ("g_out", _c_vp),
+                ("gs_out", _c_vp), ("out_scales", _c_vp)]
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib_status_string(status)} ({status})")
+
+
+_LIB = None
+SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
+           "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_get_device_status")
+
+
+def lib():
+    """The loaded C library (ctypes), with argument types declared."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"NVFP4 CUDA library not built ({LIB_PATH} missing): "
+            "run `python -m nvfp4_w4a4_quantized_02_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.nvfp4_status_string.restype = ctypes.c_char_p
+    L.nvfp4_status_string.argtypes = [ctypes.c_int]
+    L.nvfp4_scale_bytes.restype = ctypes.c_size_t
+    L.nvfp4_scale_bytes.argtypes = [_c_i64, _c_i64]
+    L.nvfp4_global_scale.restype = ctypes.c_int
+    L.nvfp4_global_scale.argtypes = [_c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp]
+    L.nvfp4_quantize.restype = ctypes.c_int
+    L.nvfp4_quantize.argtypes = [_c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp]
+    L.nvfp4_quantize_rows.restype = ctypes.c_int
+    L.nvfp4_quantize_rows.argtypes = [_c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_vp]
+    L.nvfp4_linear.restype = ctypes.c_int
+    L.nvfp4_linear.argtypes = [ctypes.POINTER(Operand), _c_vp, ctypes.POINTER(Operand),
+                               ctypes.POINTER(Segment), ctypes.c_int, ctypes.c_int,
+                               ctypes.POINTER(EpilogueParams), _c_vp, ctypes.c_int, _c_i64, _c_vp]
+    L.nvfp4_get_device_status.restype = ctypes.c_int
+    L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    _LIB = L
+    return L
+
+
+def _lib_status_string(status: int) -> str:
+    try:
+        return lib().nvfp4_status_string(status).decode()
+    except Exception:  # pragma: no cover - message formatting only
+        return "status"
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise NVFP4Error(status, what)
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return _c_vp(s.cuda_stream)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def scale_bytes(rows: int, cols: int) -> int:
+    return int(lib().nvfp4_scale_bytes(rows, cols))
+
+
+@dataclass
+class NVFP4Tensor:
+    """A quantised [rows x cols] matrix: packed codes, swizzled scales, global scale (device)."""
+    codes: "torch.Tensor"   # uint8 [rows, cols/2]
+    scales: "torch.Tensor"  # uint8 [scale_bytes(rows, cols)]
+    gs: "torch.Tensor"      # float32 [1]
+    rows: int
+    cols: int
+
+
+def global_scale(x, out=None, stream=None):
+    """gs = 2688 / max|x| of a 2-D BF16 CUDA tensor, as a float32 [1] device tensor."""
+    import torch
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_cuda
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().nvfp4_global_scale(_c_vp(x.data_ptr()), x.shape[0], x.shape[1], x.stride(0),
+                                    _c_vp(out.data_ptr()), _stream(stream)), "nvfp4_global_scale")
+    return out
+
+
+def quantize(x, gs=None, codes=None, scales=None, stream=None) -> NVFP4Tensor:
+    """NVFP4-quantise a 2-D BF16 CUDA tensor (row stride x.stride(0), unit column stride).
+
+    ``gs``: float32 [1] device tensor (static scale); None computes it from x first.
+    """
+    import torch
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_cuda and x.stride(1) == 1
+    rows, cols = x.shape
+    if gs is None:
+        gs = global_scale(x, stream=stream)
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(scale_bytes(rows, cols), 1), dtype=torch.uint8, device=x.device)
+    _check(lib().nvfp4_quantize(_c_vp(x.data_ptr()), rows, cols, x.stride(0), _c_vp(gs.data_ptr()),
+                                _c_vp(codes.data_ptr()), _c_vp(scales.data_ptr()), _stream(stream)),
+           "nvfp4_quantize")
+    return NVFP4Tensor(codes, scales, gs, rows, cols)
+
+
+def quantize_fused(parts, gs_list=None, stream=None):
+    """Quantise the modules of a fused weight, each with its own global scale, into one
+    NVFP4 weight.  ``parts``: list of 2-D BF16 CUDA tensors (same cols).
+
+    Returns ``(NVFP4Tensor, segments)`` with segments ``[(n_begin, n_end, gs), ...]``.
+    """
+    import torch
+    cols = parts[0].shape[1]
+    total = sum(p.shape[0] for p in parts)
+    dev = parts[0].device
+    codes = torch.empty((total, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(scale_bytes(total, cols), dtype=torch.uint8, device=dev)
+    segs, n0 = [], 0
+    for i, p in enumerate(parts):
+        assert p.dtype == torch.bfloat16 and p.shape[1] == cols and p.stride(1) == 1
+        gs = gs_list[i] if gs_list is not None else global_scale(p, stream=stream)
+        _check(lib().nvfp4_quantize_rows(_c_vp(p.data_ptr()), p.shape[0], cols, p.stride(0),
+                                         _c_vp(gs.data_ptr()), _c_vp(codes.data_ptr()),
+                                         _c_vp(scales.data_ptr()), n0, total, _stream(stream)),
+               "nvfp4_quantize_rows")
+        segs.append((n0, n0 + p.shape[0], gs))
+        n0 += p.shape[0]
+    return NVFP4Tensor(codes, scales, segs[0][2], total, cols), segs
+
+
+def linear(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None, epilogue: str = "none",
+           out_dtype: str = "bf16", out=None, ldo: Optional[int] = None, gates: Optional[dict] = None,
+           gs_out=None, out_scales=None, stream=None):
+    """Fused W4A4 linear ``epilogue(A @ W^T / (gs_a * gs_w[seg]))``.
+
+    segments: list of ``(n_begin, n_end, gs_w_tensor)``; default one segment with ``w.gs``.
+    gates (gdn_gates): dict with beta_begin, alpha_begin, n_heads, A_log, dt_bias
+    [, beta_out, g_out] (float32 device tensors).
+    out_dtype "nvfp4" returns an NVFP4Tensor quantised with ``gs_out``.
+    """
+    import torch
+    L = lib()
+    M, K = a.rows, a.cols
+    N = w.rows
+    if segments is None:
+        segments = [(0, N, w.gs)]
+    if len(segments) > MAX_SEGMENTS:
+        raise ValueError("too many segments")
+    segs = (Segment * len(segments))(*[Segment(int(n0), int(n1), _ptr(g)) for n0, n1, g in segments])
+    nout = N // 2 if epilogue == "silu_mul" else N
+    ep = EpilogueParams()
+    if epilogue == "gdn_gates":
+        g = gates or {}
+        ep.beta_begin, ep.alpha_begin, ep.n_heads = int(g["beta_begin"]), int(g["alpha_begin"]), int(g["n_heads"])
+        ep.A_log, ep.dt_bias = _ptr(g["A_log"]), _ptr(g["dt_bias"])
+        ep.beta_out, ep.g_out = _ptr(g.get("beta_out")), _ptr(g.get("g_out"))
+    result = None
+    if out_dtype == "nvfp4":
+        if gs_out is None:
+            raise ValueError("nvfp4 output needs gs_out")
+        if out is None:
+            out = torch.empty((M, nout // 2), dtype=torch.uint8, device=a.codes.device)
+        if out_scales is None:
+            out_scales = torch.empty(scale_bytes(M, nout), dtype=torch.uint8, device=a.codes.device)
+        ep.gs_out, ep.out_scales = _ptr(gs_out), _ptr(out_scales)
+        ldo = 0
+        result = NVFP4Tensor(out, out_scales, gs_out, M, nout)
+    else:
+        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+        if out is None:
+            out = torch.empty((M, nout), dtype=dt, device=a.codes.device)
+        ldo = out.stride(0) if ldo is None else ldo
+        result = out
+    A = Operand(a.codes.data_ptr(), a.scales.data_ptr(), M, K)
+    W = Operand(w.codes.data_ptr(), w.scales.data_ptr(), N, w.cols)
+    _check(L.nvfp4_linear(ctypes.byref(A), _c_vp(a.gs.data_ptr()), ctypes.byref(W), segs, len(segments),
+                          EPILOGUES[epilogue], ctypes.byref(ep), _c_vp(out.data_ptr()), OUT_KINDS[out_dtype],
+                          int(ldo), _stream(stream)), "nvfp4_linear")
+    return result
+
+
+def device_status() -> int:
+    """Read and clear the device status word (synchronises the device)."""
+    code = ctypes.c_int(0)
+    _check(lib().nvfp4_get_device_status(ctypes.byref(code)), "nvfp4_get_device_status")
+    return code.value

@@ -1,0 +1,292 @@
+// C ABI of the NVFP4 W4A4 linear library (declared in include/nvfp4.h):
+// argument validation, TMA descriptor creation and kernel launches.
+// Everything runs asynchronously on the caller's stream; nothing is allocated.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "nvfp4.h"
+#include "quantize.cuh"
+#include "gemm.cuh"
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+  bool gemm_attr = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Current device, checked to be an sm_100 part; fills `info`.
+nvfp4_status_t current_device(DeviceInfo **info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    d.ok = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.init = true;
+  }
+  if (!d.ok) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+  if (!d.gemm_attr) {
+    if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
+        cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    d.gemm_attr = true;
+  }
+  *info = &d;
+  return NVFP4_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map of packed codes [rows x K/2] bytes: 128-byte x 128-row boxes with the
+// 128-byte swizzle (the smem layout the MMA descriptors describe); rows beyond
+// `rows` read as zero.
+bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline nvfp4_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+}  // namespace
+
+extern "C" {
+
+const char *nvfp4_status_string(int s) {
+  switch (s) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "NVFP4_ERR_UNSUPPORTED_SHAPE";
+    case NVFP4_ERR_MISALIGNED: return "NVFP4_ERR_MISALIGNED";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
+    case NVFP4_ERR_UNSUPPORTED_DEVICE: return "NVFP4_ERR_UNSUPPORTED_DEVICE";
+    default: return "NVFP4_ERR_UNKNOWN";
+  }
+}
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows < 1 || cols < 16 || cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return 0;
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t kb_pad = (cols / 16 + 3) / 4 * 4;
+  return static_cast<size_t>(rows_pad * kb_pad);
+}
+
+nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *gs_out,
+                                  nvfp4_stream_t stream) {
+  if (!x_bf16 || !gs_out || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x_bf16, 16) || ld % 8 != 0 || !aligned(gs_out, 4)) return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(gs_out, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  AmaxArgs a;
+  a.x = static_cast<const uint16_t *>(x_bf16);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.chunks_per_row = (cols + 63) / 64;
+  a.amax_bits = reinterpret_cast<unsigned int *>(gs_out);
+  const int64_t chunks = rows * a.chunks_per_row;
+  const int64_t want = (chunks + kQuantThreads - 1) / kQuantThreads;
+  const int grid = static_cast<int>(want < int64_t(dev->sms) * 8 ? want : int64_t(dev->sms) * 8);
+  amax_kernel<<<grid, kQuantThreads, 0, s>>>(a);
+  global_scale_finalize_kernel<<<1, 1, 0, s>>>(gs_out);
+  return launch_status();
+}
+
+nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, const float *gs,
+                                   uint8_t *codes, uint8_t *scales, int64_t row_offset, int64_t total_rows,
+                                   nvfp4_stream_t stream) {
+  if (!x_bf16 || !gs || !codes || !scales || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+  if (row_offset < 0 || total_rows < row_offset + rows) return NVFP4_ERR_INVALID_ARG;
+  if (cols < 16 || cols % 16 != 0 || total_rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x_bf16, 16) || ld % 8 != 0 || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(gs, 4))
+    return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  QuantArgs a;
+  a.x = static_cast<const uint16_t *>(x_bf16);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.gs = gs;
+  a.codes = codes;
+  a.scales = scales;
+  a.row_offset = row_offset;
+  const bool last = row_offset + rows == total_rows;
+  a.rows_cover = last ? (total_rows + 127) / 128 * 128 - row_offset : rows;
+  a.kb_atoms = (cols + 63) / 64;
+  const int64_t chunks = a.rows_cover * a.kb_atoms;
+  const int64_t grid = (chunks + kQuantThreads - 1) / kQuantThreads;
+  if (grid > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  quantize_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
+nvfp4_status_t nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, const float *gs,
+                              uint8_t *codes, uint8_t *scales, nvfp4_stream_t stream) {
+  return nvfp4_quantize_rows(x_bf16, rows, cols, ld, gs, codes, scales, 0, rows, stream);
+}
+
+nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
+                            const nvfp4_segment_t *segs, int nseg, int epilogue, const nvfp4_epilogue_params_t *ep,
+                            void *out, int out_kind, int64_t ldo, nvfp4_stream_t stream) {
+  using namespace gemm;
+  if (!A || !W || !gs_a || !segs || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!A->codes || !A->scales || !W->codes || !W->scales) return NVFP4_ERR_INVALID_ARG;
+  if (A->rows < 1 || W->rows < 1 || A->K < 1 || A->K != W->K) return NVFP4_ERR_INVALID_ARG;
+  if (epilogue < NVFP4_EPI_NONE || epilogue > NVFP4_EPI_GDN_GATES) return NVFP4_ERR_INVALID_ARG;
+  if (out_kind < NVFP4_OUT_BF16 || out_kind > NVFP4_OUT_NVFP4) return NVFP4_ERR_INVALID_ARG;
+  if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  const int64_t M = A->rows, N = W->rows, K = A->K;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (K % BK != 0 || N % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  // segments: sorted, disjoint, 16-aligned, covering [0, N)
+  int64_t expect = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (!segs[i].gs_w || !aligned(segs[i].gs_w, 4)) return NVFP4_ERR_INVALID_ARG;
+    if (segs[i].n_begin != expect || segs[i].n_end <= segs[i].n_begin) return NVFP4_ERR_INVALID_ARG;
+    if (segs[i].n_begin % 16 != 0 || segs[i].n_end % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    expect = segs[i].n_end;
+  }
+  if (expect != N) return NVFP4_ERR_INVALID_ARG;
+  int64_t Nout = N;
+  if (epilogue == NVFP4_EPI_SILU_MUL) {
+    if (N % (2 * 128) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    Nout = N / 2;
+  }
+  if (epilogue == NVFP4_EPI_GDN_GATES) {
+    if (!ep || !ep->A_log || !ep->dt_bias || ep->n_heads < 1) return NVFP4_ERR_INVALID_ARG;
+    const int64_t h = ep->n_heads;
+    if (ep->beta_begin < 0 || ep->beta_begin + h > N || ep->alpha_begin < 0 || ep->alpha_begin + h > N)
+      return NVFP4_ERR_INVALID_ARG;
+    if (ep->beta_begin < ep->alpha_begin + h && ep->alpha_begin < ep->beta_begin + h) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(ep->A_log, 4) || !aligned(ep->dt_bias, 4) || (ep->beta_out && !aligned(ep->beta_out, 4)) ||
+        (ep->g_out && !aligned(ep->g_out, 4)))
+      return NVFP4_ERR_MISALIGNED;
+  }
+  if (out_kind == NVFP4_OUT_NVFP4) {
+    if (!ep || !ep->gs_out || !ep->out_scales) return NVFP4_ERR_INVALID_ARG;
+    if (Nout % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(out, 16) || !aligned(ep->out_scales, 16) || !aligned(ep->gs_out, 4)) return NVFP4_ERR_MISALIGNED;
+  } else {
+    const int64_t elem = out_kind == NVFP4_OUT_BF16 ? 2 : 4;
+    if (ldo < Nout) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || (ldo * elem) % 16 != 0) return NVFP4_ERR_MISALIGNED;
+  }
+  if (!aligned(A->codes, 16) || !aligned(W->codes, 16) || !aligned(A->scales, 16) || !aligned(W->scales, 16) ||
+      !aligned(gs_a, 4))
+    return NVFP4_ERR_MISALIGNED;
+
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+
+  CUtensorMap tmA, tmB;
+  if (!make_codes_map(&tmA, A->codes, M, K) || !make_codes_map(&tmB, W->codes, N, K)) return NVFP4_ERR_CUDA;
+
+  Params p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.Nout = static_cast<int>(Nout);
+  p.mode = epilogue;
+  p.out_kind = out_kind;
+  p.m_tiles = static_cast<int>((M + BM - 1) / BM);
+  p.n_tiles = epilogue == NVFP4_EPI_SILU_MUL ? static_cast<int>(Nout / 128) : static_cast<int>((N + BN - 1) / BN);
+  p.k_tiles = static_cast<int>(K / BK);
+  p.up_row0 = static_cast<int>(Nout);
+  p.kb_atoms = K / 64;
+  p.sfa = A->scales;
+  p.sfb = W->scales;
+  p.w_rows_pad = static_cast<int>((N + 127) / 128 * 128);
+  p.gs_a = gs_a;
+  p.nseg = nseg;
+  for (int i = 0; i < nseg; ++i) {
+    p.seg[i].n_begin = static_cast<int>(segs[i].n_begin);
+    p.seg[i].n_end = static_cast<int>(segs[i].n_end);
+    p.seg[i].gs_w = segs[i].gs_w;
+  }
+  p.out = out;
+  p.ldo = ldo;
+  p.beta_begin = p.alpha_begin = -1;
+  p.n_heads = 0;
+  if (epilogue == NVFP4_EPI_GDN_GATES) {
+    p.beta_begin = static_cast<int>(ep->beta_begin);
+    p.alpha_begin = static_cast<int>(ep->alpha_begin);
+    p.n_heads = static_cast<int>(ep->n_heads);
+    p.A_log = ep->A_log;
+    p.dt_bias = ep->dt_bias;
+    p.beta_out = ep->beta_out;
+    p.g_out = ep->g_out;
+  }
+  if (out_kind == NVFP4_OUT_NVFP4) {
+    p.gs_out = ep->gs_out;
+    p.out_scales = ep->out_scales;
+    p.out_kb_atoms = Nout / 64;
+  }
+  const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles;
+  if (tiles > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
+  gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(tmA, tmB, p);
+  return launch_status();
+}
+
+nvfp4_status_t nvfp4_get_device_status(int *code) {
+  if (!code) return NVFP4_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return NVFP4_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  *code = v;
+  return NVFP4_OK;
+}
+
+}  // extern "C"

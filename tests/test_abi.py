@@ -1,0 +1,84 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every declared entry
+point, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_w4a4_quantized_02_b200 as nv
+from nvfp4_w4a4_quantized_02_b200 import build as nvbuild
+from oracle import layout
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    assert set(syms) == set(nv.SYMBOLS), syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+    out = os.popen(f"nm -D --defined-only {nv.LIB_PATH}").read()
+    exported = set(re.findall(r" T (\w+)", out))
+    assert set(declared_symbols()) <= exported
+    # nothing else of ours leaks out of the library
+    assert {s for s in exported if s.startswith("nvfp4")} == set(declared_symbols())
+
+
+def test_scale_bytes_matches_layout_reading(L):
+    for rows, cols in [(1, 16), (128, 64), (129, 80), (300, 512), (32768, 5120), (8192, 17408)]:
+        assert nv.scale_bytes(rows, cols) == layout.scale_bytes(rows, cols)
+    assert nv.scale_bytes(0, 64) == 0 and nv.scale_bytes(4, 8) == 0 and nv.scale_bytes(4, 24) == 0
+
+
+def test_status_strings(L):
+    names = [L.nvfp4_status_string(i).decode() for i in range(7)]
+    assert names[0] == "NVFP4_OK" and names[5] == "NVFP4_ERR_DEVICE_TIMEOUT"
+    assert L.nvfp4_status_string(99).decode() == "NVFP4_ERR_UNKNOWN"
+
+
+def test_invalid_arguments_rejected_without_launch(L):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # never dereferenced: validation fails first
+    assert L.nvfp4_quantize(None, 4, 64, 64, fake, fake, fake, None) == 1
+    assert L.nvfp4_quantize(fake, 4, 24, 24, fake, fake, fake, None) == 2      # cols % 16
+    assert L.nvfp4_quantize(vp((1 << 20) + 2), 4, 64, 64, fake, fake, fake, None) == 3  # x misaligned
+    assert L.nvfp4_quantize(fake, 4, 64, 60, fake, fake, fake, None) == 1      # ld < cols
+    assert L.nvfp4_global_scale(fake, 4, 64, 64, None, None) == 1
+    A = nv.Operand(1 << 20, 1 << 21, 128, 512)
+    W = nv.Operand(1 << 22, 1 << 23, 256, 512)
+    segs = (nv.Segment * 1)(nv.Segment(0, 256, 1 << 24))
+    ep = nv.EpilogueParams()
+    call = lambda A_, W_, s, n, epi, okind, ldo, out=fake: L.nvfp4_linear(
+        ctypes.byref(A_), fake, ctypes.byref(W_), s, n, epi, ctypes.byref(ep), out, okind, ldo, None)
+    A_badk = nv.Operand(1 << 20, 1 << 21, 128, 320)
+    W_badk = nv.Operand(1 << 22, 1 << 23, 256, 320)
+    assert call(A_badk, W_badk, segs, 1, 0, 0, 256) == 2               # K % 256
+    assert call(A, W, segs, 0, 0, 0, 256) == 1                         # no segment
+    assert call(A, W, segs, 1, 7, 0, 256) == 1                         # unknown epilogue
+    assert call(A, W, segs, 1, 0, 9, 256) == 1                         # unknown output kind
+    bad = (nv.Segment * 2)(nv.Segment(0, 128, 1 << 24), nv.Segment(144, 256, 1 << 24))
+    assert call(A, W, bad, 2, 0, 0, 256) == 1                          # gap in segments
+    odd = (nv.Segment * 2)(nv.Segment(0, 120, 1 << 24), nv.Segment(120, 256, 1 << 24))
+    assert call(A, W, odd, 2, 0, 0, 256) == 2                          # bound % 16
+    assert call(A, W, segs, 1, 0, 0, 100) == 1                         # ldo < N
+    assert call(A, W, segs, 1, 0, 0, 256, out=vp((1 << 20) + 8)) == 3  # out misaligned
+    assert call(A, W, segs, 1, 2, 0, 256) == 1                         # gates without params
+    assert call(A, W, segs, 1, 0, 2, 0) == 1                           # nvfp4 out without gs_out
+    W_odd = nv.Operand(1 << 22, 1 << 23, 384, 512)
+    segs384 = (nv.Segment * 1)(nv.Segment(0, 384, 1 << 24))
+    assert call(A, W_odd, segs384, 1, 1, 0, 192) == 2                  # silu_mul needs N % 256
