@@ -86,7 +86,11 @@ def _nearest_even(a: np.ndarray, table: np.ndarray) -> np.ndarray:
     d_lo = np.abs(a - table[lo])
     d_hi = np.abs(table[hi] - a)
     pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
-    return np.where(pick_hi, hi, lo).astype(np.int64)
+    idx = np.where(pick_hi, hi, lo)
+    # at or beyond the largest entry the result saturates to it (decided by comparison,
+    # not by distances, which stop being distinguishable in FP64 for huge inputs)
+    idx = np.where(a >= table[-1], len(table) - 1, idx)
+    return idx.astype(np.int64)
 
 
 def e2m1_encode(v) -> np.ndarray:

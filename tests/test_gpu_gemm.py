@@ -163,11 +163,13 @@ def test_gdn_gates_epilogue(nv):
     assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= 1e-3
     o = bf16_to_f64(out)
     assert_gemm_close(out[:, :512], y[:, :512])
-    # gated columns of the BF16 output hold the gate values (<= 1 BF16 ulp of the oracle)
+    # gated columns of the BF16 output hold the gate values: within the gates' 1e-3
+    # absolute tolerance plus one BF16 rounding step of the value
     for got, ref in ((o[:, 512:528], beta_ref), (o[:, 528:544], g_ref)):
-        rb = oracle.round_to_bf16(ref)
-        ulp = np.ldexp(1.0, np.frexp(np.abs(rb))[1] - 8)
-        assert np.all(np.abs(got - rb) <= ulp * 1.0001)
+        ulp = np.ldexp(1.0, np.frexp(np.abs(ref))[1] - 8)
+        err = np.abs(got - ref)
+        bad = err > 1e-3 + ulp
+        assert not bad.any(), (np.argwhere(bad)[:4], got[bad][:4], ref[bad][:4])
 
 
 def test_silu_mul_epilogue_and_requant(nv):

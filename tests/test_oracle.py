@@ -5,10 +5,10 @@ format definition (golden file), an exhaustive search, an exact special case or
 a mathematical identity, chosen so that a dropped term, a wrong sign, a wrong
 index or a transposed operand in the oracle fails at least one test.
 """
-import itertools
 import json
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -35,11 +35,12 @@ def test_e2m1_decode_matches_value_set(facts):
 
 
 def _brute_e2m1(v):
-    """Nearest of the 8 magnitudes by exhaustive search; ties to the even code."""
-    mags = [abs(x) for x in json.load(open(GOLDEN))["e2m1_values_by_code"][:8]]
+    """Nearest of the 8 magnitudes by exhaustive search in exact rational arithmetic;
+    ties to the even code."""
+    mags = [Fraction(abs(x)) for x in json.load(open(GOLDEN))["e2m1_values_by_code"][:8]]
     best = None
     for code, m in enumerate(mags):
-        d = abs(abs(v) - m)
+        d = abs(abs(Fraction(v)) - m)
         if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
             best = (d, code)
     code = best[1]
@@ -52,7 +53,8 @@ def test_e2m1_encode_brute_force_sweep():
     # dense sweep over [-8, 8] including every midpoint and every representable value
     mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
     grid = np.unique(np.concatenate([np.linspace(-8, 8, 4097), mids, -mids,
-                                     [6.0, 7.0, 1e6, -1e6, 0.2499999, 0.2500001]]))
+                                     [6.0, 7.0, 1e6, -1e6, 0.2499999, 0.2500001,
+                                      1e18, -2.7e18, 3e38, -3e38, 1e300]]))
     got = oracle.e2m1_encode(grid)
     want = np.array([_brute_e2m1(float(v)) for v in grid], dtype=np.uint8)
     assert np.array_equal(got, want)
@@ -92,11 +94,13 @@ def test_e4m3_known_values(facts):
     assert np.all(np.diff(fin) > 0)
 
 
-_E4M3_TABLE = [float(oracle.e4m3_decode(c)) for c in range(0x7F)]
+_E4M3_TABLE = [Fraction(float(oracle.e4m3_decode(c))) for c in range(0x7F)]
 
 
 def _brute_e4m3(s):
+    """Nearest finite E4M3 by exhaustive search in exact rational arithmetic; ties to even."""
     best = None
+    s = Fraction(s)
     for code, val in enumerate(_E4M3_TABLE):
         d = abs(s - val)
         if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
@@ -109,7 +113,8 @@ def test_e4m3_encode_brute_force():
     fin = oracle.e4m3_decode(np.arange(0x7F))
     mids = (fin[1:] + fin[:-1]) / 2
     s = np.concatenate([rng.uniform(0, 500, 3000), np.exp(rng.uniform(-14, 6.5, 3000)),
-                        mids, fin, [448.0, 449.0, 464.0, 480.0, 1e9, 0.0, 2.0 ** -10, 2.0 ** -11]])
+                        mids, fin, [448.0, 449.0, 464.0, 480.0, 1e9, 0.0, 2.0 ** -10, 2.0 ** -11,
+                                    2.0e20, 3.0e38]])
     s = s.astype(np.float32).astype(np.float64)
     got = oracle.e4m3_encode(s)
     want = np.array([_brute_e4m3(float(x)) for x in s], dtype=np.uint8)
