@@ -1,11 +1,20 @@
 #!/usr/bin/env python
 """Benchmark of the NVFP4 W4A4 linear hot path on B200.
 
-One JSON line on stdout (rank 0).  Default workload: the MLP block at 32768 prefill
-tokens (X BF16 [32768 x 5120] -> global scale -> NVFP4 quantise -> fused gate|up
-GEMM [2 x 17408 rows, separate global scales] with SiLU*mul and NVFP4
-re-quantisation in the epilogue -> down-projection GEMM [5120 x 17408] -> BF16).
-Other workloads: ``--workload quantize|gdn|linear``.
+One JSON line on stdout (rank 0).  Workloads (``--workload``):
+
+* ``mlp`` (default): the MLP block at 32768 prefill tokens.  X BF16 [32768 x 5120]
+  -> global scale -> NVFP4 quantise -> fused gate|up GEMM [2 x 17408 rows, separate
+  global scales] with SiLU*mul and NVFP4 re-quantisation in the epilogue ->
+  down-projection GEMM [5120 x 17408] -> BF16.
+* ``quantize``: activation quantisation of X BF16 [32768 x 5120] (Student-t, 8 hot
+  channels) with a static global scale -> packed E2M1 + swizzled E4M3 scales.
+* ``gdn``: GDN fused input projection, X [8192 x 5120] -> one NVFP4 GEMM over
+  q|k|v|z|beta|alpha (12352 rows, six global scales) with the gate epilogue.
+* ``linear``: the small single linear, X [128 x 1024] x W [1024 x 1024]^T.
+* ``sweep``: all 496 linears of the 64-layer hybrid model (48 GDN layers x 2 GEMMs,
+  16 attention layers x 2 GEMMs with q|k|v fused, 64 MLPs x 2 GEMMs with gate|up
+  fused), each fed by the NVFP4 quantiser, at ``--M`` prefill tokens.
 
 Multi-GPU (torchrun): every rank runs the same workload on its own GPU with its own
 inputs (independent token batches, weak scaling); no collective touches the data
@@ -17,6 +26,7 @@ same workload on the host cores, as the reference arm.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -31,6 +41,7 @@ sys.path.insert(0, ROOT)
 METRIC = "NVFP4 W4A4 linear TFLOPS & % of B200 dense FP4 peak; quantise GB/s vs HBM"
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
 
 
 # ----------------------------------------------------------------- helpers
@@ -110,22 +121,83 @@ def dist_env():
     return ws, rank, local
 
 
-# --------------------------------------------------------------- workloads
-class Workload:
-    """Inputs resident on the device plus a ``step()`` that runs the hot path once."""
-    name = ""
-    unit = "TFLOP/s"
-
-    def flops(self) -> float:
-        return 0.0
-
-
-def _dev_bits(bits):
-    import numpy as np
-    import torch
-    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+def sources_hash(files):
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "nvfp4_w4a4_quantized_02_b200", "csrc")
+    for fn in files:
+        with open(os.path.join(d, fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
+def load_traffic(key):
+    """DRAM bytes per launch of ``key`` (``kernel@workload``) from the committed ncu
+    summary ``profiles/traffic.json``, or None when the kernel's sources changed since."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            ent = json.load(f).get(key)
+        if ent and ent.get("csrc_sha256") == sources_hash(ent["sources"]):
+            return ent["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class KernelTimer:
+    """CUDA events around individual launches on the launching (current) stream.
+
+    ``with tm("key"):`` brackets one launch; ``summary()`` gives per key the number
+    of launches and their summed / average duration over all recorded steps.
+    """
+
+    def __init__(self, torch):
+        self.torch = torch
+        self.recs = []
+
+    def __call__(self, key):
+        return _KernelSpan(self, key)
+
+    def summary(self):
+        out = {}
+        for key, e0, e1 in self.recs:
+            d = out.setdefault(key, {"launches": 0, "ms_total": 0.0})
+            d["launches"] += 1
+            d["ms_total"] += e0.elapsed_time(e1)
+        for d in out.values():
+            d["ms_avg"] = d["ms_total"] / d["launches"]
+        return out
+
+
+class _KernelSpan:
+    def __init__(self, tm, key):
+        self.tm, self.key = tm, key
+
+    def __enter__(self):
+        ev = self.tm.torch.cuda.Event
+        self.e0, self.e1 = ev(enable_timing=True), ev(enable_timing=True)
+        self.e0.record()
+
+    def __exit__(self, *exc):
+        self.e1.record()
+        self.tm.recs.append((self.key, self.e0, self.e1))
+        return False
+
+
+class _NoTimer:
+    def __call__(self, key):
+        return self
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+NO_TIMER = _NoTimer()
+
+
+# --------------------------------------------------------- synthetic inputs
 def _gpu_student_t(rows, cols, seed, hot=8, hot_factor=100.0):
     """Student-t(3) activations generated on the device (seeded torch RNG), BF16.
 
@@ -149,20 +221,90 @@ def _gpu_student_t(rows, cols, seed, hot=8, hot_factor=100.0):
     return out
 
 
+def _gpu_outliers(rows, cols, seed, frac=1e-3, factor=50.0):
+    """N(0,1) activations with ``frac`` of the entries (seeded permutation) x ``factor``, BF16."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    x = torch.randn((rows, cols), generator=g, device="cuda")
+    n = int(round(frac * rows * cols))
+    if n:
+        idx = torch.randperm(rows * cols, generator=g, device="cuda")[:n]
+        x.view(-1)[idx] *= factor
+    return x.to(torch.bfloat16)
+
+
 def _gpu_normal(rows, cols, seed, std):
     import torch
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
-    return (torch.randn((rows, cols), generator=g, device="cuda") * std).to(torch.bfloat16)
+    out = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda")
+    step = max(1, (1 << 27) // cols)
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        out[r0:r1] = (torch.randn((r1 - r0, cols), generator=g, device="cuda") * std).to(torch.bfloat16)
+    return out
+
+
+GDN_SEGMENTS = (("q", 2048, 1.0), ("k", 2048, 2.0), ("v", 4096, 4.0), ("z", 4096, 8.0),
+                ("beta", 32, 16.0), ("alpha", 32, 1.0))
+
+
+def _gdn_weight(nv, K, seed):
+    """Fused GDN in-projection weight q|k|v|z|beta|alpha, each segment its own global scale."""
+    parts = [_gpu_normal(n, K, seed + i, 0.02 * m) for i, (_, n, m) in enumerate(GDN_SEGMENTS)]
+    w, segs = nv.quantize_fused(parts)
+    del parts
+    return w, segs
+
+
+def _gdn_gate_tensors(torch, M, seed):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    a_log = torch.randn(32, generator=g, device="cuda")
+    dt_bias = torch.randn(32, generator=g, device="cuda")
+    beta = torch.empty((M, 32), dtype=torch.float32, device="cuda")
+    gate = torch.empty((M, 32), dtype=torch.float32, device="cuda")
+    n = sum(n for _, n, _ in GDN_SEGMENTS)
+    return dict(beta_begin=n - 64, alpha_begin=n - 32, n_heads=32, A_log=a_log, dt_bias=dt_bias,
+                beta_out=beta, g_out=gate)
+
+
+# --------------------------------------------------------------- workloads
+class Workload:
+    """Inputs resident on the device plus a ``step(tm)`` that runs the hot path once.
+
+    ``unit``: "TFLOP/s" or "GB/s"; ``work()``: FLOPs or bytes per step (the
+    algorithmic count); ``dominant``: (timer key, work per launch, bound, label).
+    """
+    name = ""
+    unit = "TFLOP/s"
+    flush_l2 = False
+    l2_note = ""
+    launches_per_step = 0
+    x = None      # the step's input (refreshed from host memory in the e2e run)
+    out = None    # the step's result (read back in the e2e run)
+
+    def work(self) -> float:
+        raise NotImplementedError
+
+    def config(self) -> dict:
+        return {}
+
+    def cpu_sample(self):
+        """One bounded CPU-oracle sample of this workload: (work in the metric's base unit, seconds)."""
+        raise NotImplementedError
+
+    cpu_sample_note = ""
 
 
 class MLPBlock(Workload):
-    """MLP block, 32768 tokens: quantise X, gate|up GEMM + SiLU*mul + NVFP4 requant, down GEMM."""
-    name = "mlp_block_m32768_h5120_i17408"
+    """MLP block: quantise X, gate|up GEMM + SiLU*mul + NVFP4 requant, down GEMM."""
 
     def __init__(self, nv, M=32768, H=5120, I=17408, seed=0):
         import torch
         self.nv, self.M, self.H, self.I = nv, M, H, I
+        self.name = f"mlp_block_m{M}_h{H}_i{I}"
         self.x = _gpu_student_t(M, H, seed)
         wg = _gpu_normal(I, H, seed + 1, 0.02)
         wu = _gpu_normal(I, H, seed + 2, 0.04)
@@ -186,37 +328,363 @@ class MLPBlock(Workload):
         del h16
         torch.cuda.synchronize()
         self.launches_per_step = 5  # amax, finalize, quantize, gate|up GEMM, down GEMM
+        self.f_gu = 2.0 * M * (2 * I) * H
+        self.f_d = 2.0 * M * H * I
+        self.l2_note = (f"inputs larger than L2 (X {M * H * 2 / 1e6:.0f} MB, H {M * I * 0.5625 / 1e6:.0f} MB, "
+                        f"out {M * H * 2 / 1e6:.0f} MB per step)")
+        self.dominant = ("gemm_gate_up", self.f_gu, "tensor",
+                         "gemm_kernel (gate|up, SiLU*mul, NVFP4 requant epilogue)")
+        self.phases = {"global_scale": ("GB/s", 2.0 * M * H), "quantize": ("GB/s", 2.5625 * M * H),
+                       "gemm_gate_up": ("TFLOP/s", self.f_gu), "gemm_down": ("TFLOP/s", self.f_d)}
 
-    def flops(self):
-        return 2.0 * self.M * (2 * self.I) * self.H + 2.0 * self.M * self.H * self.I
+    def work(self):
+        return self.f_gu + self.f_d
 
-    def step(self, ev=None, x=None):
+    def config(self):
+        return {"M": self.M, "hidden": self.H, "intermediate": self.I,
+                "step": "global_scale+quantize(X) -> gate|up GEMM (SiLU*mul, NVFP4 requant) -> down GEMM (BF16)"}
+
+    def step(self, tm=NO_TIMER, x=None):
         nv = self.nv
         x = self.x if x is None else x
-        nv.global_scale(x, out=self.gs_x)
-        if ev: ev["q0"].record()
-        xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
-        if ev: ev["q1"].record()
-        hq = nv.linear(xq, self.w_gu, segments=self.seg_gu, epilogue="silu_mul", out_dtype="nvfp4",
-                       gs_out=self.gs_h, out=self.h_codes, out_scales=self.h_scales)
-        if ev: ev["g1"].record()
-        nv.linear(hq, self.w_d, out_dtype="bf16", out=self.out)
-        if ev: ev["g2"].record()
+        with tm("global_scale"):
+            nv.global_scale(x, out=self.gs_x)
+        with tm("quantize"):
+            xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
+        with tm("gemm_gate_up"):
+            hq = nv.linear(xq, self.w_gu, segments=self.seg_gu, epilogue="silu_mul", out_dtype="nvfp4",
+                           gs_out=self.gs_h, out=self.h_codes, out_scales=self.h_scales)
+        with tm("gemm_down"):
+            nv.linear(hq, self.w_d, out_dtype="bf16", out=self.out)
         return self.out
 
-    def kernel_report(self, times_ms, peaks):
-        q_bytes = self.M * self.H * 2.5625
-        f_gu = 2.0 * self.M * (2 * self.I) * self.H
-        f_d = 2.0 * self.M * self.H * self.I
-        rep = {
-            "quantize": {"ms": times_ms["quantize"], "GB/s": q_bytes / times_ms["quantize"] / 1e6},
-            "gemm_gate_up_silu_requant": {"ms": times_ms["gemm1"], "TFLOP/s": f_gu / times_ms["gemm1"] / 1e9},
-            "gemm_down": {"ms": times_ms["gemm2"], "TFLOP/s": f_d / times_ms["gemm2"] / 1e9},
-        }
-        rep["quantize"]["frac_hbm"] = rep["quantize"]["GB/s"] / peaks["hbm_gbs"]
-        return rep
+    cpu_sample_note = ("MLP-block sample (32 token rows, 256 intermediate channels, K=5120; global scale + "
+                       "quantise + gate|up + SiLU*mul + requant + down); numpy FP64 oracle")
+
+    def cpu_sample(self):
+        return cpu_mlp_sample()
 
 
+class QuantizeOnly(Workload):
+    """Activation quantisation with a static (calibrated) global scale."""
+    unit = "GB/s"
+
+    def __init__(self, nv, M=32768, K=5120, seed=0):
+        import torch
+        self.nv, self.M, self.K = nv, M, K
+        self.name = f"quantize_m{M}_k{K}"
+        self.x = _gpu_student_t(M, K, seed)
+        self.gs = nv.global_scale(self.x)
+        self.gs_dyn = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        self.scales = torch.empty(nv.scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+        self.out = self.codes
+        self.launches_per_step = 1
+        self.bytes = 2.5625 * M * K
+        self.l2_note = f"input larger than L2 (X {M * K * 2 / 1e6:.0f} MB)"
+        self.dominant = ("quantize", self.bytes, "hbm", "quantize_kernel (static global scale)")
+        self.phases = {"quantize": ("GB/s", self.bytes)}
+        torch.cuda.synchronize()
+
+    def work(self):
+        return self.bytes
+
+    def config(self):
+        return {"M": self.M, "K": self.K, "gs": "static (calibrated once from amax)",
+                "bytes_per_element": 2.5625}
+
+    def step(self, tm=NO_TIMER, x=None):
+        x = self.x if x is None else x
+        with tm("quantize"):
+            self.nv.quantize(x, self.gs, codes=self.codes, scales=self.scales)
+        return self.codes
+
+    def extra(self, torch):
+        """Dynamic mode (amax pass + finalize + quantise), timed separately after the main region."""
+        nv = self.nv
+        for _ in range(3):
+            nv.global_scale(self.x, out=self.gs_dyn)
+            nv.quantize(self.x, self.gs_dyn, codes=self.codes, scales=self.scales)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 10
+        s.record()
+        for _ in range(n):
+            nv.global_scale(self.x, out=self.gs_dyn)
+            nv.quantize(self.x, self.gs_dyn, codes=self.codes, scales=self.scales)
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / n
+        b = 4.5625 * self.M * self.K
+        return {"dynamic_gs": {"ms": ms, "GB/s": b / ms / 1e6, "bytes_per_element": 4.5625}}
+
+    cpu_sample_note = "quantise of 64 rows x 5120 (Student-t, static gs); numpy oracle"
+
+    def cpu_sample(self):
+        import oracle
+        import synth
+        x = synth.bf16_to_f32(synth.student_t_activations(64, self.K, seed=0))
+        gs = oracle.global_scale(x)
+        t0 = time.perf_counter()
+        oracle.quantize(x, gs)
+        return 2.5625 * x.size, time.perf_counter() - t0
+
+
+class GDNInProj(Workload):
+    """GDN fused input projection: quantise X, one GEMM over six segments + gate epilogue."""
+
+    def __init__(self, nv, M=8192, K=5120, seed=0):
+        import torch
+        self.nv, self.M, self.K = nv, M, K
+        self.N = sum(n for _, n, _ in GDN_SEGMENTS)
+        self.name = f"gdn_inproj_m{M}_n{self.N}_k{K}"
+        self.x = _gpu_outliers(M, K, seed)
+        self.w, self.segs = _gdn_weight(nv, K, seed + 1)
+        self.gates = _gdn_gate_tensors(torch, M, seed + 100)
+        self.gs_x = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.xq_codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        self.xq_scales = torch.empty(nv.scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((M, self.N), dtype=torch.bfloat16, device="cuda")
+        self.flops = 2.0 * M * self.N * K
+        self.launches_per_step = 4
+        self.l2_note = (f"per-step working set {(M * K * 2.5625 + self.N * K * 0.5625 + M * self.N * 2) / 1e6:.0f} MB "
+                        "> L2 (X, its codes, W, BF16 out)")
+        self.dominant = ("gemm", self.flops, "tensor", "gemm_kernel (6 segments, GDN gate epilogue)")
+        self.phases = {"global_scale": ("GB/s", 2.0 * M * K), "quantize": ("GB/s", 2.5625 * M * K),
+                       "gemm": ("TFLOP/s", self.flops)}
+        torch.cuda.synchronize()
+
+    def work(self):
+        return self.flops
+
+    def config(self):
+        return {"M": self.M, "N": self.N, "K": self.K,
+                "segments": "q 2048 | k 2048 | v 4096 | z 4096 | beta 32 | alpha 32",
+                "step": "global_scale+quantize(X) -> fused GEMM (per-segment alpha, sigmoid beta, "
+                        "-exp(A_log)*softplus(a+dt_bias)) -> BF16 + FP32 gates"}
+
+    def step(self, tm=NO_TIMER, x=None):
+        nv = self.nv
+        x = self.x if x is None else x
+        with tm("global_scale"):
+            nv.global_scale(x, out=self.gs_x)
+        with tm("quantize"):
+            xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
+        with tm("gemm"):
+            nv.linear(xq, self.w, segments=self.segs, epilogue="gdn_gates", gates=self.gates,
+                      out_dtype="bf16", out=self.out)
+        return self.out
+
+    cpu_sample_note = ("GDN in-proj sample: 32 token rows x 320 weight rows (64 each of q/k/v/z + 32 beta + "
+                       "32 alpha), K=5120; quantise X + fused linear + gates; numpy FP64 oracle")
+
+    def cpu_sample(self):
+        return cpu_gdn_sample(self.K)
+
+
+class SmallLinear(Workload):
+    """Single small W4A4 linear (dynamic activation scale): launch-latency bound."""
+    flush_l2 = True
+
+    def __init__(self, nv, M=128, N=1024, K=1024, seed=0):
+        import torch
+        self.nv, self.M, self.N, self.K = nv, M, N, K
+        self.name = f"linear_m{M}_n{N}_k{K}"
+        self.x = _gpu_outliers(M, K, seed)
+        self.w = nv.quantize(_gpu_normal(N, K, seed + 1, 0.02))
+        self.gs_x = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.xq_codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        self.xq_scales = torch.empty(nv.scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        self.flops = 2.0 * M * N * K
+        self.launches_per_step = 4
+        self.l2_note = "L2 flushed (256 MB write) between timed steps; per-step device time summed"
+        self.dominant = ("gemm", self.flops, "tensor", "gemm_kernel (1 segment, BF16 out)")
+        self.phases = {"global_scale": ("GB/s", 2.0 * M * K), "quantize": ("GB/s", 2.5625 * M * K),
+                       "gemm": ("TFLOP/s", self.flops)}
+        torch.cuda.synchronize()
+
+    def work(self):
+        return self.flops
+
+    def config(self):
+        return {"M": self.M, "N": self.N, "K": self.K,
+                "step": "global_scale+quantize(X) -> GEMM -> BF16"}
+
+    def step(self, tm=NO_TIMER, x=None):
+        nv = self.nv
+        x = self.x if x is None else x
+        with tm("global_scale"):
+            nv.global_scale(x, out=self.gs_x)
+        with tm("quantize"):
+            xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
+        with tm("gemm"):
+            nv.linear(xq, self.w, out_dtype="bf16", out=self.out)
+        return self.out
+
+    cpu_sample_note = "the whole linear (128 x 1024 x 1024): quantise X + dequantise-then-FP64 matmul"
+
+    def cpu_sample(self):
+        import oracle
+        import synth
+        x = synth.bf16_to_f32(synth.outlier_activations(self.M, self.K, seed=0))
+        w = synth.bf16_to_f32(synth.gaussian_weights(self.N, self.K, seed=1))
+        gw = oracle.global_scale(w)
+        cw, sw = oracle.quantize(w, gw)
+        t0 = time.perf_counter()
+        gx = oracle.global_scale(x)
+        cx, sx = oracle.quantize(x, gx)
+        oracle.linear(cx, sx, gx, cw, sw, [(0, self.N, gw)])
+        return self.flops, time.perf_counter() - t0
+
+
+class HybridSweep(Workload):
+    """The 496 linears of the 64-layer hybrid model, each fed by the NVFP4 quantiser.
+
+    Layers 4j..4j+2 are GDN, 4j+3 attention (48 + 16); every layer has an MLP.
+    GDN: in-proj 5120 -> 12352 (q|k|v|z|beta|alpha, gate epilogue) + out 4096 -> 5120.
+    Attention: q|k|v 5120 -> 6144|1024|1024 fused + o 6144 -> 5120.
+    MLP: gate|up 5120 -> 2 x 17408 (SiLU*mul, NVFP4 requant) + down 17408 -> 5120.
+    Linear count: 48 x 5 + 16 x 4 + 64 x 3 = 496 (fused GEMMs count their modules).
+    The inputs of the out / o projections stand in for the mixer outputs (the mixers
+    themselves are not linears): fixed Student-t tensors of width 4096 / 6144.
+    """
+
+    def __init__(self, nv, M=32768, seed=0):
+        import torch
+        self.nv, self.M = nv, M
+        self.name = f"hybrid_sweep_496_linears_m{M}"
+        H, I = 5120, 17408
+        dev = "cuda"
+        # activations per distinct input width, each with a static calibrated global scale
+        self.x = _gpu_student_t(M, H, seed)
+        self.x_gdn_core = _gpu_student_t(M, 4096, seed + 1)
+        self.x_attn_core = _gpu_student_t(M, 6144, seed + 2)
+        self.gs_x = nv.global_scale(self.x)
+        self.gs_gc = nv.global_scale(self.x_gdn_core)
+        self.gs_ac = nv.global_scale(self.x_attn_core)
+
+        def qbuf(rows, cols):
+            return (torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                    torch.empty(nv.scale_bytes(rows, cols), dtype=torch.uint8, device=dev))
+        self.qx = qbuf(M, H)
+        self.qgc = qbuf(M, 4096)
+        self.qac = qbuf(M, 6144)
+        self.hq = qbuf(M, I)
+        self.out_gdn = torch.empty((M, 12352), dtype=torch.bfloat16, device=dev)
+        self.out_qkv = torch.empty((M, 8192), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        self.gates = _gdn_gate_tensors(torch, M, seed + 100)
+        self.layers = []
+        s = seed + 1000
+        for li in range(64):
+            L = {}
+            if li % 4 == 3:
+                qkv = [_gpu_normal(6144, H, s, 0.02), _gpu_normal(1024, H, s + 1, 0.02),
+                       _gpu_normal(1024, H, s + 2, 0.02)]
+                L["qkv"] = nv.quantize_fused(qkv)
+                del qkv
+                L["o"] = nv.quantize(_gpu_normal(H, 6144, s + 3, 0.02))
+            else:
+                L["in"] = _gdn_weight(nv, H, s)
+                L["out"] = nv.quantize(_gpu_normal(H, 4096, s + 10, 0.02))
+            gu = [_gpu_normal(I, H, s + 20, 0.02), _gpu_normal(I, H, s + 21, 0.02)]
+            L["gu"] = nv.quantize_fused(gu)
+            del gu
+            L["down"] = nv.quantize(_gpu_normal(H, I, s + 22, 0.02))
+            self.layers.append(L)
+            s += 100
+        torch.cuda.synchronize()
+        # static global scale of the MLP hidden state, calibrated on layer 0
+        xq = nv.quantize(self.x, self.gs_x, codes=self.qx[0], scales=self.qx[1])
+        w, segs = self.layers[0]["gu"]
+        h16 = nv.linear(xq, w, segments=segs, epilogue="silu_mul", out_dtype="bf16")
+        self.gs_h = nv.global_scale(h16)
+        del h16
+        torch.cuda.synchronize()
+        per_tok = (48 * 2 * (12352 * H + H * 4096) + 16 * 2 * (8192 * H + H * 6144)
+                   + 64 * 2 * (2 * I * H + H * I))
+        self.flops = float(per_tok) * M
+        self.f_gu = 2.0 * M * 2 * I * H
+        self.launches_per_step = 48 * 4 + 16 * 4 + 64 * 3
+        self.packed_bytes = sum(t.codes.numel() + t.scales.numel()
+                                for L in self.layers for v in L.values()
+                                for t in ([v[0]] if isinstance(v, tuple) else [v]))
+        self.l2_note = f"weights {self.packed_bytes / 2**30:.2f} GiB packed, streamed once per step (> L2)"
+        self.dominant = ("gemm_gate_up", self.f_gu, "tensor",
+                         "gemm_kernel (MLP gate|up, SiLU*mul, NVFP4 requant epilogue)")
+        self.phases = {"quantize": ("GB/s", 2.5625 * M * (128 * H + 48 * 4096 + 16 * 6144)),
+                       "gemm_gdn_in": ("TFLOP/s", 48 * 2.0 * M * 12352 * H),
+                       "gemm_gdn_out": ("TFLOP/s", 48 * 2.0 * M * H * 4096),
+                       "gemm_attn_qkv": ("TFLOP/s", 16 * 2.0 * M * 8192 * H),
+                       "gemm_attn_o": ("TFLOP/s", 16 * 2.0 * M * H * 6144),
+                       "gemm_gate_up": ("TFLOP/s", 64 * self.f_gu),
+                       "gemm_down": ("TFLOP/s", 64 * 2.0 * M * H * I)}
+
+    def work(self):
+        return self.flops
+
+    def config(self):
+        return {"M": self.M, "layers": "48 GDN + 16 attention, 64 MLP", "linears": 496,
+                "gemm_launches_per_step": 256, "packed_weight_gib": round(self.packed_bytes / 2**30, 3),
+                "step": "per layer: quantise(input) -> fused NVFP4 GEMM(s) with the layer's epilogue"}
+
+    def step(self, tm=NO_TIMER, x=None):
+        nv = self.nv
+        x = self.x if x is None else x
+        qx = None
+        for li, L in enumerate(self.layers):
+            with tm("quantize"):
+                qx = nv.quantize(x, self.gs_x, codes=self.qx[0], scales=self.qx[1])
+            if "qkv" in L:
+                w, segs = L["qkv"]
+                with tm("gemm_attn_qkv"):
+                    nv.linear(qx, w, segments=segs, out_dtype="bf16", out=self.out_qkv)
+                with tm("quantize"):
+                    qc = nv.quantize(self.x_attn_core, self.gs_ac, codes=self.qac[0], scales=self.qac[1])
+                with tm("gemm_attn_o"):
+                    nv.linear(qc, L["o"], out_dtype="bf16", out=self.out)
+            else:
+                w, segs = L["in"]
+                with tm("gemm_gdn_in"):
+                    nv.linear(qx, w, segments=segs, epilogue="gdn_gates", gates=self.gates, out_dtype="bf16",
+                              out=self.out_gdn)
+                with tm("quantize"):
+                    qc = nv.quantize(self.x_gdn_core, self.gs_gc, codes=self.qgc[0], scales=self.qgc[1])
+                with tm("gemm_gdn_out"):
+                    nv.linear(qc, L["out"], out_dtype="bf16", out=self.out)
+            with tm("quantize"):
+                qx = nv.quantize(x, self.gs_x, codes=self.qx[0], scales=self.qx[1])
+            w, segs = L["gu"]
+            with tm("gemm_gate_up"):
+                hq = nv.linear(qx, w, segments=segs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=self.gs_h,
+                               out=self.hq[0], out_scales=self.hq[1])
+            with tm("gemm_down"):
+                nv.linear(hq, L["down"], out_dtype="bf16", out=self.out)
+        return self.out
+
+    cpu_sample_note = ("one sampled MLP block and one sampled GDN in-proj (32 token rows, 256-320 weight rows, "
+                       "full K), FLOP-weighted; numpy FP64 oracle")
+
+    def cpu_sample(self):
+        f1, s1 = cpu_mlp_sample()
+        f2, s2 = cpu_gdn_sample(5120)
+        return f1 + f2, s1 + s2
+
+
+WORKLOADS = {"mlp": MLPBlock, "quantize": QuantizeOnly, "gdn": GDNInProj, "linear": SmallLinear,
+             "sweep": HybridSweep}
+
+
+def make_workload(args, nv):
+    cls = WORKLOADS[args.workload]
+    kw = {}
+    if args.M:
+        kw["M"] = args.M
+    return cls(nv, **kw)
+
+
+# ---------------------------------------------------------------- GPU arm
 def run_ours(args, ws, rank):
     import torch
     import nvfp4_w4a4_quantized_02_b200 as nv
@@ -225,17 +693,21 @@ def run_ours(args, ws, rank):
         build.build()
     if ws > 1:
         torch.distributed.barrier()
+    nv.lib()
     peaks, peak_src = load_peaks()
-    wl = MLPBlock(nv)
+    wl = make_workload(args, nv)
     stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda") if wl.flush_l2 else None
 
-    # warm-up
     for _ in range(args.warmup):
         wl.step()
+        if flush is not None:
+            flush.zero_()
     torch.cuda.synchronize()
 
-    evn = ["q0", "q1", "g1", "g2"]
-    evs = [{k: torch.cuda.Event(enable_timing=True) for k in evn} for _ in range(args.steps)]
+    tm = KernelTimer(torch)
+    steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
@@ -247,57 +719,79 @@ def run_ours(args, ws, rank):
     time.sleep(0.3)
     start.record(stream)
     for i in range(args.steps):
-        wl.step(evs[i])
+        steps[i][0].record(stream)
+        wl.step(tm)
+        steps[i][1].record(stream)
+        if flush is not None:
+            flush.zero_()
     stop.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    elapsed_ms = start.elapsed_time(stop)
+    if flush is not None:
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in steps)
+    else:
+        elapsed_ms = start.elapsed_time(stop)
     if ws > 1:
         t = torch.tensor([elapsed_ms], device="cuda")
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         elapsed_ms = float(t.item())
         torch.distributed.barrier()
-    per = {"quantize": [], "gemm1": [], "gemm2": []}
-    for e in evs:
-        per["quantize"].append(e["q0"].elapsed_time(e["q1"]))
-        per["gemm1"].append(e["q1"].elapsed_time(e["g1"]))
-        per["gemm2"].append(e["g1"].elapsed_time(e["g2"]))
-    times = {k: sum(v) / len(v) for k, v in per.items()}
 
-    # end to end through the public API with host buffers
-    e2e = run_e2e(wl, args, torch)
+    ksum = tm.summary()
+    kernels = {}
+    for key, (unit, amount) in wl.phases.items():
+        if key not in ksum:
+            continue
+        ms = ksum[key]["ms_total"] / args.steps
+        d = {"launches_per_step": ksum[key]["launches"] // args.steps, "ms_per_step": round(ms, 5)}
+        if unit == "GB/s":
+            d["GB/s"] = round(amount / ms / 1e6, 1)
+            d["frac_hbm"] = round(d["GB/s"] / peaks["hbm_gbs"], 4)
+        else:
+            d["TFLOP/s"] = round(amount / ms / 1e9, 1)
+            d["frac_fp4_peak"] = round(d["TFLOP/s"] / (peaks["bf16_tflops_sustained"] * FP4_OVER_BF16), 4)
+        kernels[key] = d
 
+    key, per_launch, bound, label = wl.dominant
+    avg_ms = ksum[key]["ms_avg"]
+    if bound == "hbm":
+        achieved = per_launch / avg_ms / 1e6
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        note = f"{peak_src} hbm_gbs (copy bandwidth)"
+    else:
+        achieved = per_launch / avg_ms / 1e9
+        peak, unit = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16, "TFLOP/s"
+        note = f"{peak_src} bf16_tflops_sustained x {FP4_OVER_BF16} (nominal FP4/BF16 ratio)"
+    roof = {"kernel": label, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": load_traffic(f"{key}@{wl.name}"),
+            "avg_launch_ms": round(avg_ms, 5), "work_per_launch": per_launch, "peak_note": note}
+
+    e2e = run_e2e(wl, args, torch, flush)
     ms = elapsed_ms / args.steps
-    value = ws * wl.flops() / (ms * 1e-3) / 1e12
-    rep = wl.kernel_report(times, peaks)
-    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
-    g = rep["gemm_gate_up_silu_requant"]
-    roof = {"kernel": "gemm_kernel (gate|up, SiLU*mul, NVFP4 requant epilogue)", "bound": "tensor",
-            "achieved": g["TFLOP/s"], "peak": fp4_peak, "unit": "TFLOP/s", "frac": g["TFLOP/s"] / fp4_peak,
-            "traffic": load_traffic("gemm_mlp_gate_up"),
-            "peak_note": f"{peak_src} bf16_tflops_sustained x {FP4_OVER_BF16} (nominal FP4/BF16 ratio)"}
-    for k in rep:
-        if "TFLOP/s" in rep[k]:
-            rep[k]["frac_fp4_peak"] = rep[k]["TFLOP/s"] / fp4_peak
+    if wl.unit == "GB/s":
+        value = ws * wl.work() / (ms * 1e-3) / 1e9
+    else:
+        value = ws * wl.work() / (ms * 1e-3) / 1e12
+    cfg = {"workload": wl.name, **wl.config(),
+           "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU", "l2": wl.l2_note}
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "nvfp4(e2m1+e4m3)->fp32 acc", "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.M, "hidden": wl.H, "intermediate": wl.I,
-                   "step": "global_scale+quantize(X) -> gate|up GEMM (SiLU*mul, NVFP4 requant) -> down GEMM (BF16)",
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (X 335 MB, H 285 MB, out 335 MB per step)"},
-        "roofline": roof, "kernels": rep, "e2e": e2e, "gpu_launches": wl.launches_per_step * args.steps,
-        "clocks": clocks, "peaks_source": peak_src,
+        "vs_baseline": None, "dtype": "nvfp4(e2m1+e4m3)->fp32 acc" if wl.unit != "GB/s" else "bf16->nvfp4",
+        "data": "synthetic", "config": cfg, "roofline": roof, "kernels": kernels, "e2e": e2e,
+        "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks, "peaks_source": peak_src,
     }
+    if hasattr(wl, "extra"):
+        line["kernels"].update(wl.extra(torch))
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args)
+        line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(wl, args, torch):
-    """Same step through the public API with host buffers: pinned H2D of X, the step, D2H of the output."""
+def run_e2e(wl, args, torch, flush):
+    """The same step through the public API with host buffers: pinned H2D of the step's
+    input, the step, D2H of its result, all inside the timed region."""
     stream = torch.cuda.current_stream()
     x_host = wl.x.cpu().pin_memory()
     out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
@@ -307,40 +801,25 @@ def run_e2e(wl, args, torch):
         x_dev.copy_(x_host, non_blocking=True)
         out_host.copy_(wl.step(x=x_dev), non_blocking=True)
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(n):
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
         x_dev.copy_(x_host, non_blocking=True)
         out_host.copy_(wl.step(x=x_dev), non_blocking=True)
-    e.record(stream)
+        b.record(stream)
+        if flush is not None:
+            flush.zero_()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / n
-    return {"value": round(wl.flops() / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": out_host.numel() * 2,
+    ms = sum(a.elapsed_time(b) for a, b in evs) / n
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
+    return {"value": round(wl.work() / (ms * 1e-3) / scale, 2), "unit": wl.unit,
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
             "ms_per_step": round(ms, 4), "steps": n}
 
 
-def load_traffic(key):
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
-    import hashlib
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    try:
-        with open(path) as f:
-            d = json.load(f)
-        h = hashlib.sha256()
-        for fn in sorted(os.listdir(os.path.join(ROOT, "nvfp4_w4a4_quantized_02_b200", "csrc"))):
-            with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_02_b200", "csrc", fn), "rb") as f:
-                h.update(f.read())
-        ent = d.get(key)
-        if ent and ent.get("csrc_sha256") == h.hexdigest():
-            return ent["bytes_per_launch"]
-    except Exception:
-        pass
-    return None
-
-
 # ---------------------------------------------------------------- CPU oracle
-def cpu_sample_step(rows=32, cols_h=256, K=5120):
+def cpu_mlp_sample(rows=32, cols_h=256, K=5120):
     """The MLP block restated by the oracle on a bounded sample: ``rows`` token rows, a
     slice of ``cols_h`` intermediate channels (gate and up), K=5120 in, the down
     projection over those channels for all 5120 outputs.  Returns (flops, seconds)."""
@@ -369,41 +848,92 @@ def cpu_sample_step(rows=32, cols_h=256, K=5120):
     return flops, dt
 
 
-def cpu_baseline(args, budget_s=12.0):
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    flops, secs, n = 0.0, 0.0, 0
+def cpu_gdn_sample(K=5120, rows=32):
+    """GDN in-projection on a bounded sample: ``rows`` tokens, 64 rows of each of q/k/v/z
+    plus the 32 beta and 32 alpha rows, each segment with its own global scale."""
+    import numpy as np
+    import oracle
+    import synth
+    x = synth.bf16_to_f32(synth.outlier_activations(rows, K, seed=0))
+    names = [("q", 64), ("k", 64), ("v", 64), ("z", 64), ("beta", 32), ("alpha", 32)]
+    ws = synth.segmented_weights(names, K, seed=1, multipliers=synth.GDN_INPROJ_MULTIPLIERS)
+    cs, ss, segs, n0 = [], [], [], 0
+    for _, wb in ws:
+        w = synth.bf16_to_f32(wb)
+        g = oracle.global_scale(w)
+        c, s = oracle.quantize(w, g)
+        cs.append(c), ss.append(s), segs.append((n0, n0 + w.shape[0], g))
+        n0 += w.shape[0]
+    a_log, dt_bias = synth.gdn_gate_params(32)
+    t0 = time.perf_counter()
+    gx = oracle.global_scale(x)
+    cx, sx = oracle.quantize(x, gx)
+    y = oracle.linear(cx, sx, gx, np.concatenate(cs), np.concatenate(ss), segs)
+    oracle.gdn_gates(y[:, 256:288], y[:, 288:320], a_log, dt_bias)
+    return 2.0 * rows * n0 * K, time.perf_counter() - t0
+
+
+def _cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    work, secs, n = 0.0, 0.0, 0
     t_end = time.perf_counter() + budget_s
     while time.perf_counter() < t_end or n == 0:
-        f, s = cpu_sample_step()
-        flops += f
+        w, s = wl.cpu_sample()
+        work += w
         secs += s
         n += 1
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} x MLP-block sample (32 token rows, 256 intermediate channels, K=5120; "
-                      "global scale + quantise + gate|up + SiLU*mul + requant + down); numpy FP64 oracle"}
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
+    return {"value": work / secs / scale, "unit": wl.unit, "cores": _cores(), "kind": "oracle",
+            "sample": f"{n} x {wl.cpu_sample_note}"}
+
+
+class _CpuOnly:
+    """Workload descriptor for the reference arm (no GPU objects)."""
+
+    def __init__(self, args):
+        cls = WORKLOADS[args.workload]
+        self.cls = cls
+        self.unit = cls.unit
+        self.cpu_sample_note = cls.cpu_sample_note
+        obj = object.__new__(cls)
+        obj.M = args.M or {"mlp": 32768, "quantize": 32768, "gdn": 8192, "linear": 128, "sweep": 32768}[args.workload]
+        obj.K = {"quantize": 5120, "gdn": 5120, "linear": 1024}.get(args.workload, 5120)
+        obj.N = {"linear": 1024, "gdn": 12352}.get(args.workload, 0)
+        obj.flops = 2.0 * obj.M * obj.N * obj.K
+        self.obj = obj
+        self.name = {"mlp": f"mlp_block_m{obj.M}_h5120_i17408", "quantize": f"quantize_m{obj.M}_k5120",
+                     "gdn": f"gdn_inproj_m{obj.M}_n12352_k5120", "linear": f"linear_m{obj.M}_n1024_k1024",
+                     "sweep": f"hybrid_sweep_496_linears_m{obj.M}"}[args.workload]
+
+    def cpu_sample(self):
+        return self.cls.cpu_sample(self.obj)
 
 
 def run_reference(args, ws, rank):
     if rank != 0:
         return
+    wl = _CpuOnly(args)
     t0 = time.perf_counter()
     for _ in range(args.warmup):
-        cpu_sample_step()
-    flops, secs = 0.0, 0.0
+        wl.cpu_sample()
+    work, secs = 0.0, 0.0
     for _ in range(args.steps):
-        f, s = cpu_sample_step()
-        flops += f
+        w, s = wl.cpu_sample()
+        work += w
         secs += s
-    value = flops / secs / 1e12
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+    scale = 1e9 if wl.unit == "GB/s" else 1e12
+    value = work / secs / scale
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
             "data": "synthetic",
-            "config": {"workload": MLPBlock.name, "sample": "32 rows x 256 intermediate channels per step"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": "MLP-block sample per step (32 rows, 256 channels, K=5120)"},
-            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "config": {"workload": wl.name, "sample": wl.cpu_sample_note},
+            "cpu_baseline": {"value": value, "unit": wl.unit, "cores": _cores(), "kind": "oracle",
+                             "sample": f"per step: {wl.cpu_sample_note}"},
+            "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": round(time.perf_counter() - t0, 2)}
     print(json.dumps(line), flush=True)
 
@@ -414,6 +944,8 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mlp")
+    ap.add_argument("--M", type=int, default=0, help="token rows (default: the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     ws, rank, local = dist_env()

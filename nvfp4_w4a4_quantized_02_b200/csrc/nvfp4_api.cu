@@ -21,7 +21,8 @@ struct DeviceInfo {
   bool init = false;
   bool ok = false;
   int sms = 0;
-  bool gemm_attr = false;
+  bool attrs = false;
+  int quant_ctas_per_sm = 1;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -46,11 +47,17 @@ nvfp4_status_t current_device(DeviceInfo **info) {
     d.init = true;
   }
   if (!d.ok) return NVFP4_ERR_UNSUPPORTED_DEVICE;
-  if (!d.gemm_attr) {
+  if (!d.attrs) {
     if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes) !=
+            cudaSuccess)
       return NVFP4_ERR_CUDA;
-    d.gemm_attr = true;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel, kQThreads, kQSmemBytes) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    d.quant_ctas_per_sm = occ < 1 ? 1 : occ;
+    d.attrs = true;
   }
   *info = &d;
   return NVFP4_OK;
@@ -84,6 +91,21 @@ bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t 
   cuuint32_t box[2] = {128, 128};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor map of a BF16 matrix [rows x cols] with row stride ld elements: 64-column x
+// 128-row boxes (128 bytes per box row) with the 128-byte swizzle; coordinates
+// outside the matrix read as zero.
+bool make_bf16_map(CUtensorMap *m, const void *x, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kQTileCols), static_cast<cuuint32_t>(kQTileRows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -132,12 +154,12 @@ nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols
   a.rows = rows;
   a.cols = cols;
   a.ld = ld;
-  a.chunks_per_row = (cols + 63) / 64;
   a.amax_bits = reinterpret_cast<unsigned int *>(gs_out);
-  const int64_t chunks = rows * a.chunks_per_row;
-  const int64_t want = (chunks + kQuantThreads - 1) / kQuantThreads;
-  const int grid = static_cast<int>(want < int64_t(dev->sms) * 8 ? want : int64_t(dev->sms) * 8);
-  amax_kernel<<<grid, kQuantThreads, 0, s>>>(a);
+  const int64_t vecs = rows * (cols / 8);
+  const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
+  const int64_t cap = int64_t(dev->sms) * 8;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
+  amax_kernel<<<grid, kAmaxThreads, 0, s>>>(a);
   global_scale_finalize_kernel<<<1, 1, 0, s>>>(gs_out);
   return launch_status();
 }
@@ -152,22 +174,24 @@ nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t col
     return NVFP4_ERR_MISALIGNED;
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;
+  CUtensorMap tmX;
+  if (!make_bf16_map(&tmX, x_bf16, rows, cols, ld)) return NVFP4_ERR_CUDA;
   QuantArgs a;
-  a.x = static_cast<const uint16_t *>(x_bf16);
-  a.rows = rows;
-  a.cols = cols;
-  a.ld = ld;
   a.gs = gs;
   a.codes = codes;
   a.scales = scales;
+  a.rows = rows;
+  a.cols = cols;
   a.row_offset = row_offset;
   const bool last = row_offset + rows == total_rows;
-  a.rows_cover = last ? (total_rows + 127) / 128 * 128 - row_offset : rows;
+  a.own_end = last ? (total_rows + 127) / 128 * 128 : row_offset + rows;
+  a.code_ld = cols / 2;
   a.kb_atoms = (cols + 63) / 64;
-  const int64_t chunks = a.rows_cover * a.kb_atoms;
-  const int64_t grid = (chunks + kQuantThreads - 1) / kQuantThreads;
-  if (grid > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  quantize_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  a.tile_r0 = row_offset / 128;
+  a.n_tiles = ((a.own_end + 127) / 128 - a.tile_r0) * a.kb_atoms;
+  const int64_t cap = int64_t(dev->sms) * dev->quant_ctas_per_sm;
+  const int grid = static_cast<int>(a.n_tiles < cap ? a.n_tiles : cap);
+  quantize_kernel<<<grid, kQThreads, kQSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(tmX, a);
   return launch_status();
 }
 

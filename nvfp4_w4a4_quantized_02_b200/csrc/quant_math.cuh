@@ -11,22 +11,38 @@
 
 namespace nvfp4 {
 
+// E4M3 block-scale byte of a block whose maximum magnitude is `amax`.
+__device__ __forceinline__ uint32_t block_scale_byte(float amax, float gs) {
+  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+  return cvt_e4m3x2(0.0f, s) & 0xFFu;
+}
+
+// Block scale from the block's amax: returns the E4M3 byte and sets `inv`, the
+// factor that maps the block onto the E2M1 grid (0 when the scale is 0).
+__device__ __forceinline__ uint32_t block_scale(float amax, float gs, float &inv) {
+  const uint32_t sf = block_scale_byte(amax, gs);
+  inv = sf == 0 ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(sf));
+  return sf;
+}
+
+// Eight values -> eight E2M1 codes (element i in nibble i).
+__device__ __forceinline__ uint32_t encode8(const float *x, float inv) {
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[i], inv);
+  return cvt_e2m1x8(v);
+}
+
 // x[16] -> E4M3 scale byte (returned) and 16 E2M1 codes in two words (element i in
 // nibble i%8 of word i/8).
 __device__ __forceinline__ uint32_t quantize16(const float (&x)[16], float gs, uint32_t &c0, uint32_t &c1) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-  const uint32_t sf = cvt_e4m3x2(0.0f, s) & 0xFFu;
-  const float inv = sf == 0 ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(sf));
-  float v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[i], inv);
-  c0 = cvt_e2m1x8(v);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[8 + i], inv);
-  c1 = cvt_e2m1x8(v);
+  float inv;
+  const uint32_t sf = block_scale(amax, gs, inv);
+  c0 = encode8(x, inv);
+  c1 = encode8(x + 8, inv);
   return sf;
 }
 
