@@ -7,18 +7,35 @@
 // here every output column n is scaled by alpha = 1 / (gs_A * gs_W[seg(n)])),
 // section 機構② (GDN gates beta = sigmoid(b), g = -exp(A_log) * softplus(a + dt_bias)).
 //
-// Kernel structure (one persistent CTA per SM, 320 threads):
-//   warp 0      TMA producer: A / W code tiles (cp.async.bulk.tensor, 128-byte
-//               swizzle) and their scale tiles (cp.async.bulk, already in the
-//               MMA's atom layout) into a 4-stage shared-memory ring.
-//   warp 1      MMA issuer: copies the stage's scales to TMEM (tcgen05.cp), issues
-//               4 tcgen05.mma kind::mxf4nvf4 (128 x 256 x 64 each) into the TMEM
-//               accumulator, and frees the stage with tcgen05.commit.
+// Two kernels share the tile shape per CTA (128 output rows x 256 output columns,
+// K staged 256 FP4 elements = 128 bytes per row at a time) and the epilogue:
+//
+// gemm_kernel (1 CTA per tile, used when M <= 128): tcgen05.mma.cta_group::1,
+//   M = 128, N = 256; the CTA loads both 128-row halves of the B tile.
+// gemm2_kernel (a cluster of 2 CTAs per 256 x 256 tile): tcgen05.mma.cta_group::2,
+//   M = 256, N = 256, issued by the even CTA; each CTA loads its own 128 rows of A
+//   and its own 128-row half of B, so per SM the shared-memory traffic per MMA is
+//   halved against the 1-CTA kernel.  Every load signals the even CTA's stage
+//   barrier; one tcgen05.commit signals the MMA's completion to the barriers of
+//   both CTAs.  Each TMA load is a plain load of one CTA's own tile from this GPU's
+//   memory.
+//
+// Roles (one persistent CTA per SM, 352 threads):
+//   warp 0      TMA producer: code tiles (128-byte swizzle) and scale tiles (already
+//               in the MMA's 128 x 4 atom layout) into a shared-memory ring.
+//   warp 1      MMA issuer: 4 block-scaled MMAs (K = 64 each) per stage into the
+//               TMEM accumulator, then frees the stage with tcgen05.commit.
 //   warps 2..9  epilogue: tcgen05.ld the 128 x 256 FP32 accumulator (each warp a
 //               32-lane quadrant x 128 columns) into registers, hand TMEM back to the
 //               MMA warp at once, then scale / activate / store from registers.
-// Tile 128 x 256 x 256 (K in FP4 elements); output tiles are visited in groups of
-// 16 M-tiles so that concurrently running CTAs share A and W tiles in L2.
+//   warp 10     scale copier: per stage, 12 tcgen05.cp of the A and B scale atoms
+//               into that stage's TMEM scale columns, then tcgen05.commit to the
+//               MMA issuer.  Issued from their own thread, the copies of stage s+1
+//               overlap the MMAs of stage s; issued in line with the MMAs they ran
+//               in series with them and cost ~60 cycles each (measured: gate|up
+//               GEMM of the MLP block 3.26 ms -> 2.76 ms with the 1-CTA kernel).
+// Output tiles are visited in groups of 16 M-tiles so that concurrently running
+// CTAs share A and W tiles in L2.
 #pragma once
 
 #include "quant_math.cuh"
@@ -26,34 +43,51 @@
 namespace nvfp4 {
 namespace gemm {
 
-constexpr int BM = 128;
+constexpr int BM = 128;                  // output rows per CTA
 constexpr int BN = 256;
 constexpr int BK = 256;                  // FP4 elements per stage = 128 bytes per row
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK / 2;     // 16 KB
 constexpr int B_HALF_BYTES = 128 * BK / 2;
-constexpr int B_BYTES = BN * BK / 2;     // 32 KB
 constexpr int SF_ATOM = 512;             // 128 rows x 4 scale bytes
 constexpr int SFA_BYTES = 4 * SF_ATOM;   // 4 MMA k-steps
 constexpr int SFB_HALF_BYTES = 4 * SF_ATOM;
 constexpr int SFB_BYTES = 2 * SFB_HALF_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int COPY_WARP = 2 + NUM_EPI_WARPS;
+constexpr int NUM_THREADS = 32 * (COPY_WARP + 1);
 constexpr int GROUP_M = 16;
 
-// TMEM columns (allocation of 512 = the whole TMEM of the SM)
+// TMEM columns (allocation of 512 = the whole TMEM of the SM): the 256-column FP32
+// accumulator, then one set of scale columns per shared-memory stage, so that the
+// scales of stage s are rewritten only after the producer refilled stage s, which
+// needs the MMAs that read them to have completed.
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;     // 256 FP32 columns
-constexpr uint32_t SFA_COL = 256;   // 4 k-steps x 4 columns
-constexpr uint32_t SFB_COL = 272;   // 4 k-steps x 8 columns
+constexpr uint32_t ACC_COL = 0;        // 256 FP32 columns
+constexpr uint32_t SF_COL = 256;       // first scale set
+constexpr uint32_t SF_SET_COLS = 48;   // SFA: 4 k-steps x 4 columns, then SFB: 4 k-steps x 8 columns
+constexpr uint32_t SFB_OFF_COLS = 16;
+__host__ __device__ constexpr uint32_t sfa_col(int stage) { return SF_COL + SF_SET_COLS * stage; }
+__host__ __device__ constexpr uint32_t sfb_col(int stage) { return SF_COL + SF_SET_COLS * stage + SFB_OFF_COLS; }
 
-constexpr int CTRL_BYTES = 1024;
-constexpr int SMEM_A_OFF = CTRL_BYTES;
-constexpr int SMEM_B_OFF = SMEM_A_OFF + STAGES * A_BYTES;
-constexpr int SMEM_SFA_OFF = SMEM_B_OFF + STAGES * B_BYTES;
-constexpr int SMEM_SFB_OFF = SMEM_SFA_OFF + STAGES * SFA_BYTES;
-constexpr int SMEM_END = SMEM_SFB_OFF + STAGES * SFB_BYTES;
-constexpr int SMEM_BYTES = SMEM_END + 1024;  // slack to align the base to 1024
+// Shared-memory plan of a kernel whose CTA loads `b_halves` 128-row halves of B.
+template <int kStages, int kBHalves>
+struct SmemPlan {
+  static constexpr int STAGES = kStages;
+  static constexpr int B_BYTES = kBHalves * B_HALF_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int CTRL_BYTES = 1024;
+  static constexpr int A_OFF = CTRL_BYTES;
+  static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
+  static constexpr int SFA_OFF = B_OFF + STAGES * B_BYTES;
+  static constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_BYTES;
+  static constexpr int END = SFB_OFF + STAGES * SFB_BYTES;
+  static constexpr int BYTES = END + 1024;  // slack to align the base to 1024
+};
+using Plan1 = SmemPlan<4, 2>;  // 1-CTA kernel: 54 KB per stage
+using Plan2 = SmemPlan<5, 1>;  // 2-CTA kernel: 38 KB per stage
+static_assert(Plan1::BYTES <= 227 * 1024 && Plan2::BYTES <= 227 * 1024, "shared memory");
+static_assert(sfb_col(Plan1::STAGES - 1) + 32 <= TMEM_COLS && sfb_col(Plan2::STAGES - 1) + 32 <= TMEM_COLS,
+              "TMEM columns");
 
 enum Mode : int { MODE_NONE = 0, MODE_SILU_MUL = 1, MODE_GDN = 2 };
 enum OutKind : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_NVFP4 = 2 };
@@ -66,12 +100,11 @@ struct Segment {
 struct Params {
   int M, N, K, Nout;
   int mode, out_kind;
-  int m_tiles, n_tiles, k_tiles;
+  int m_tiles, n_tiles, k_tiles;  // m_tiles counts tiles of BM * (CTAs per tile) rows
   int up_row0;              // SILU_MUL: first weight row of the `up` half
   int64_t kb_atoms;         // K / 64
   const uint8_t *sfa;       // swizzled scales of A
   const uint8_t *sfb;       // swizzled scales of W
-  int w_rows_pad;           // W rows padded to 128 (rows present in sfb)
   const float *gs_a;
   int nseg;
   Segment seg[16];
@@ -87,6 +120,7 @@ struct Params {
   int64_t out_kb_atoms;
 };
 
+template <int STAGES>
 struct Ctrl {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -97,11 +131,14 @@ struct Ctrl {
   int seg_begin[16];
   int seg_end[16];
   float seg_alpha[16];
+  float inv_out[128];  // NVFP4 output: gs_out / e4m3(sf) for sf = 0..127 (0 for 0 and NaN)
+  uint64_t sf_ready[STAGES];  // the stage's scales are in TMEM (tcgen05.commit of the copier)
+  uint64_t sf_drain;
 };
-static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block too large");
+static_assert(sizeof(Ctrl<6>) <= 1024, "control block too large");
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: E2M1 A and B (format 1),
-// UE4M3 scales, K-major operands, M = 128, N = 256, dense K = 64, scale ids 0.
+// UE4M3 scales, K-major operands, dense K = 64, scale ids 0; M and N of the MMA.
 __host__ __device__ constexpr uint32_t make_idesc(int m, int n) {
   return (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
 }
@@ -126,7 +163,8 @@ __device__ __forceinline__ void b_rows(const Params &p, int nt, int &rb0, int &r
   }
 }
 
-__device__ __forceinline__ float seg_alpha(const Ctrl &c, int nseg, int n) {
+template <int STAGES>
+__device__ __forceinline__ float seg_alpha(const Ctrl<STAGES> &c, int nseg, int n) {
   float a = 0.0f;
   for (int s = 0; s < nseg; ++s)
     if (n >= c.seg_begin[s] && n < c.seg_end[s]) a = c.seg_alpha[s];
@@ -156,17 +194,25 @@ __device__ __forceinline__ void store16(const Params &p, int row, int col, const
 }
 
 // Re-quantise 64 consecutive outputs (one scale word) of one row: round to BF16,
-// then the NVFP4 block quantiser with the output's global scale.
-__device__ __forceinline__ void store64_nvfp4(const Params &p, int row, int col, const float (&y)[64],
-                                              float gs_out) {
+// then the NVFP4 block quantiser with the output's global scale (gs_out / e4m3(sf)
+// read from the CTA's table, the same FP32 division).
+__device__ __forceinline__ void store64_nvfp4(const Params &p, const float *inv_out, int row, int col,
+                                              const float (&y)[64], float gs_out) {
   uint32_t codes[8];
   uint32_t sfword = 0;
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     float x[16];
+    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(y[16 * b + i]));
-    const uint32_t sf = quantize16(x, gs_out, codes[2 * b], codes[2 * b + 1]);
+    for (int i = 0; i < 16; ++i) {
+      x[i] = __bfloat162float(__float2bfloat16_rn(y[16 * b + i]));
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+    const uint32_t sf = block_scale_byte(amax, gs_out);
+    const float inv = inv_out[sf & 127];
+    codes[2 * b] = encode8(x, inv);
+    codes[2 * b + 1] = encode8(x + 8, inv);
     sfword |= sf << (8 * b);
   }
   uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) + (int64_t)row * (p.Nout / 2) + col / 2);
@@ -175,38 +221,219 @@ __device__ __forceinline__ void store64_nvfp4(const Params &p, int row, int col,
   *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, col / 64, p.out_kb_atoms)) = sfword;
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctrl &c = *reinterpret_cast<Ctrl *>(smem);
-  uint8_t *sA = smem + SMEM_A_OFF;
-  uint8_t *sB = smem + SMEM_B_OFF;
-  uint8_t *sSFA = smem + SMEM_SFA_OFF;
-  uint8_t *sSFB = smem + SMEM_SFB_OFF;
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&c.full[s], 1);
-      mbar_init(&c.empty[s], 1);
+// GDN gates of the 64 outputs starting at column cg of one row, for the columns that
+// fall in the beta or alpha head blocks.  Kept out of line: only the N-tile holding
+// the head blocks gets here, and the unrolled epilogue stays small.
+__device__ __noinline__ void gdn_gates64(const Params &p, int row, int cg, float *y) {
+  for (int i = 0; i < 64; ++i) {
+    const int n = cg + i;
+    if (n >= p.beta_begin && n < p.beta_begin + p.n_heads) {
+      const float bt = sigmoid_f(y[i]);
+      y[i] = bt;
+      if (p.beta_out) p.beta_out[(int64_t)row * p.n_heads + (n - p.beta_begin)] = bt;
+    } else if (n >= p.alpha_begin && n < p.alpha_begin + p.n_heads) {
+      const int hh = n - p.alpha_begin;
+      const float g = -expf(__ldg(p.A_log + hh)) * softplus_f(y[i] + __ldg(p.dt_bias + hh));
+      y[i] = g;
+      if (p.g_out) p.g_out[(int64_t)row * p.n_heads + hh] = g;
     }
-    mbar_init(&c.acc_full, 1);
-    mbar_init(&c.acc_empty, NUM_EPI_WARPS);
-    mbar_init(&c.drain, 1);
-    fence_barrier_init();
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
   }
+}
+
+// TMEM -> registers for one epilogue warp: 32 lanes of quadrant q, 128 columns
+// (SILU_MUL: 64 gate columns and the matching 64 up columns).
+__device__ __forceinline__ void epilogue_load(const Params &p, uint32_t tmem, int q, int half,
+                                              uint32_t (&v)[4][32]) {
+  const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+  if (p.mode == MODE_SILU_MUL) {
+    tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 64, v[0]);
+    tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 64 + 32, v[1]);
+    tmem_ld_32x32b_x32(lane_addr + ACC_COL + 128 + half * 64, v[2]);
+    tmem_ld_32x32b_x32(lane_addr + ACC_COL + 128 + half * 64 + 32, v[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 128 + 32 * i, v[i]);
+  }
+  tmem_ld_wait();
+}
+
+// Scale / activate / store the accumulator values of one output row held by this
+// thread (columns as loaded by epilogue_load) for N-tile nt.
+template <int STAGES>
+__device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES> &c, const uint32_t (&v)[4][32],
+                                             int row, int nt, int half, float gs_out) {
+  if (row >= p.M) {
+    // padding rows of an NVFP4 output: their scale words are written as zero
+    if (p.out_kind == OUT_NVFP4) {
+      const int span = p.mode == MODE_SILU_MUL ? 64 : 128;
+      const int cbeg = p.mode == MODE_SILU_MUL ? nt * 128 + half * 64 : nt * BN + half * 128;
+      const int rows_pad = (p.M + 127) / 128 * 128;
+      if (row < rows_pad)
+        for (int cg = cbeg; cg < cbeg + span && cg < p.Nout; cg += 64)
+          *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, cg / 64, p.out_kb_atoms)) = 0u;
+    }
+    return;
+  }
+  if (p.mode == MODE_SILU_MUL) {
+    // output columns [nt*128 + half*64, +64): gate = weight row n, up = row up_row0 + n
+    const int col0 = nt * 128 + half * 64;
+    const float ag = seg_alpha(c, p.nseg, col0);
+    const float au = seg_alpha(c, p.nseg, p.up_row0 + col0);
+    float h[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float g = ag * __uint_as_float(v[i >> 5][i & 31]);
+      const float u = au * __uint_as_float(v[2 + (i >> 5)][i & 31]);
+      h[i] = __fdividef(g, 1.0f + __expf(-g)) * u;  // SiLU(g) * u
+    }
+    if (p.out_kind == OUT_NVFP4) {
+      store64_nvfp4(p, c.inv_out, row, col0, h, gs_out);
+    } else {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = h[16 * b + i];
+        store16(p, row, col0 + 16 * b, y);
+      }
+    }
+    return;
+  }
+  const int col0 = nt * BN + half * 128;
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {  // two 64-column groups
+    const int cg = col0 + 64 * hb;
+    if (cg >= p.Nout) break;
+    float y[64];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float a = seg_alpha(c, p.nseg, cg + 16 * b);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) y[16 * b + i] = a * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
+    }
+    if (p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + 64 > p.beta_begin) ||
+                               (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin))) {
+      float t[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) t[i] = y[i];
+      gdn_gates64(p, row, cg, t);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) y[i] = t[i];
+    }
+    if (p.out_kind == OUT_NVFP4) {
+      store64_nvfp4(p, c.inv_out, row, cg, y, gs_out);
+    } else {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (cg + 16 * b < p.Nout) {
+          float yy[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) yy[i] = y[16 * b + i];
+          store16(p, row, cg + 16 * b, yy);
+        }
+      }
+    }
+  }
+}
+
+// Per-CTA epilogue tables: the segments' alphas and, for an NVFP4 output, the
+// 128 possible values of gs_out / e4m3(sf).
+template <int STAGES>
+__device__ __forceinline__ void load_segments(const Params &p, Ctrl<STAGES> &c) {
   if (threadIdx.x >= 64 && threadIdx.x < 64 + p.nseg) {
     const int s = threadIdx.x - 64;
     c.seg_begin[s] = p.seg[s].n_begin;
     c.seg_end[s] = p.seg[s].n_end;
     c.seg_alpha[s] = __frcp_rn(__fmul_rn(__ldg(p.gs_a), __ldg(p.seg[s].gs_w)));
   }
+  if (p.out_kind == OUT_NVFP4 && threadIdx.x >= 128 && threadIdx.x < 256) {
+    const int sf = threadIdx.x - 128;
+    c.inv_out[sf] = (sf == 0 || sf == 127) ? 0.0f : __fdiv_rn(__ldg(p.gs_out), e4m3_to_f32(sf));
+  }
+}
+
+// Scale copier (one thread): for each stage of the CTA's run, once the stage's
+// bytes landed, copy its scale atoms into the stage's TMEM scale set and commit to
+// sf_ready[stage].  Set s is rewritten only after full[s] completed again, i.e.
+// after the producer refilled stage s, which waited for the MMAs that read set s.
+template <int STAGES, bool kPair>
+__device__ __forceinline__ void copy_scales(Ctrl<STAGES> &c, uint32_t tmem, const uint8_t *sSFA,
+                                            const uint8_t *sSFB, int total) {
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int g = 0; g < total; ++g) {
+    if (!mbar_wait(&c.full[stage], phase)) break;
+    tc_fence_after();
+    const uint32_t sfa_addr = smem_u32(sSFA + stage * SFA_BYTES);
+    const uint32_t sfb_addr = smem_u32(sSFB + stage * SFB_BYTES);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint64_t da = sdesc_plain_32x16B(sfa_addr + j * SF_ATOM);
+      const uint64_t db0 = sdesc_plain_32x16B(sfb_addr + j * SF_ATOM);
+      const uint64_t db1 = sdesc_plain_32x16B(sfb_addr + SFB_HALF_BYTES + j * SF_ATOM);
+      if constexpr (kPair) {  // each CTA's scales go to its own TMEM (same addresses in both)
+        tc_cp_32x128b_x4_cg2(tmem + sfa_col(stage) + 4 * j, da);
+        tc_cp_32x128b_x4_cg2(tmem + sfb_col(stage) + 8 * j, db0);
+        tc_cp_32x128b_x4_cg2(tmem + sfb_col(stage) + 8 * j + 4, db1);
+      } else {
+        tc_cp_32x128b_x4(tmem + sfa_col(stage) + 4 * j, da);
+        tc_cp_32x128b_x4(tmem + sfb_col(stage) + 8 * j, db0);
+        tc_cp_32x128b_x4(tmem + sfb_col(stage) + 8 * j + 4, db1);
+      }
+    }
+    if constexpr (kPair) {
+      tc_commit_cg2(&c.sf_ready[stage]);
+    } else {
+      tc_commit(&c.sf_ready[stage]);
+    }
+    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+  }
+  // wait for every copy this thread issued
+  if constexpr (kPair) {
+    tc_commit_cg2(&c.sf_drain);
+  } else {
+    tc_commit(&c.sf_drain);
+  }
+  mbar_wait(&c.sf_drain, 0);
+}
+
+template <int STAGES>
+__device__ __forceinline__ void init_barriers(Ctrl<STAGES> &c, uint32_t acc_empty_count) {
+  for (int s = 0; s < STAGES; ++s) {
+    mbar_init(&c.full[s], 1);
+    mbar_init(&c.empty[s], 1);
+    mbar_init(&c.sf_ready[s], 1);
+  }
+  mbar_init(&c.acc_full, 1);
+  mbar_init(&c.acc_empty, acc_empty_count);
+  mbar_init(&c.drain, 1);
+  mbar_init(&c.sf_drain, 1);
+  fence_barrier_init();
+}
+
+// ============================================================ 1-CTA kernel
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ Params p) {
+  using P = Plan1;
+  constexpr int STAGES = P::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl<STAGES> &c = *reinterpret_cast<Ctrl<STAGES> *>(smem);
+  uint8_t *sA = smem + P::A_OFF;
+  uint8_t *sB = smem + P::B_OFF;
+  uint8_t *sSFA = smem + P::SFA_OFF;
+  uint8_t *sSFB = smem + P::SFB_OFF;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    init_barriers(c, NUM_EPI_WARPS);
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  load_segments(p, c);
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -216,6 +443,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
   const int num_tiles = p.m_tiles * p.n_tiles;
+  const int my_tiles = num_tiles > (int)blockIdx.x ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -239,12 +467,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive_expect_tx(&c.full[stage], bytes);
           const int kx = kt * (BK / 2);
           tma_load_2d(sA + stage * A_BYTES, &tmA, &c.full[stage], kx, mt * BM);
-          tma_load_2d(sB + stage * B_BYTES, &tmB, &c.full[stage], kx, rb0);
+          tma_load_2d(sB + stage * P::B_BYTES, &tmB, &c.full[stage], kx, rb0);
           bulk_load(sSFA + stage * SFA_BYTES, sfa_src + (int64_t)kt * SFA_BYTES, SFA_BYTES, &c.full[stage]);
           bulk_load(sSFB + stage * SFB_BYTES, sfb0_src + (int64_t)kt * SFB_HALF_BYTES, SFB_HALF_BYTES,
                     &c.full[stage]);
           if (second) {
-            tma_load_2d(sB + stage * B_BYTES + B_HALF_BYTES, &tmB, &c.full[stage], kx, rb1);
+            tma_load_2d(sB + stage * P::B_BYTES + B_HALF_BYTES, &tmB, &c.full[stage], kx, rb1);
             bulk_load(sSFB + stage * SFB_BYTES + SFB_HALF_BYTES, sfb1_src + (int64_t)kt * SFB_HALF_BYTES,
                       SFB_HALF_BYTES, &c.full[stage]);
           }
@@ -269,26 +497,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1;
         tc_fence_after();
         for (int kt = 0; kt < p.k_tiles; ++kt) {
-          if (!mbar_wait(&c.full[stage], phase)) { ok = false; break; }
+          if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
-          const uint32_t sfa_addr = smem_u32(sSFA + stage * SFA_BYTES);
-          const uint32_t sfb_addr = smem_u32(sSFB + stage * SFB_BYTES);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tc_cp_32x128b_x4(tmem + SFA_COL + 4 * j, sdesc_plain_32x16B(sfa_addr + j * SF_ATOM));
-            tc_cp_32x128b_x4(tmem + SFB_COL + 8 * j, sdesc_plain_32x16B(sfb_addr + j * SF_ATOM));
-            tc_cp_32x128b_x4(tmem + SFB_COL + 8 * j + 4,
-                             sdesc_plain_32x16B(sfb_addr + SFB_HALF_BYTES + j * SF_ATOM));
-          }
-          const uint64_t a_desc = sdesc_sw128_kmajor(a_addr);
-          const uint64_t b_desc = sdesc_sw128_kmajor(b_addr);
+          const uint64_t a_desc = sdesc_sw128_kmajor(smem_u32(sA + stage * A_BYTES));
+          const uint64_t b_desc = sdesc_sw128_kmajor(smem_u32(sB + stage * P::B_BYTES));
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             // advance 64 FP4 = 32 bytes along K inside the swizzle atom (+2 in 16-byte units)
-            mma_nvfp4(tmem + ACC_COL, a_desc + 2 * j, b_desc + 2 * j, idesc, tmem + SFA_COL + 4 * j,
-                      tmem + SFB_COL + 8 * j, (kt | j) != 0);
+            mma_nvfp4(tmem + ACC_COL, a_desc + 2 * j, b_desc + 2 * j, idesc, tmem + sfa_col(stage) + 4 * j,
+                      tmem + sfb_col(stage) + 8 * j, (kt | j) != 0);
           }
           tc_commit(&c.empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -299,6 +516,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(&c.drain);
       mbar_wait(&c.drain, 0);
     }
+  } else if (warp == COPY_WARP) {
+    if (lane == 0) copy_scales<STAGES, false>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles);
   } else {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
@@ -312,99 +531,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc_phase ^= 1;
       tc_fence_after();
       uint32_t v[4][32];
-      const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-      if (p.mode == MODE_SILU_MUL) {
-        tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 64, v[0]);
-        tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 64 + 32, v[1]);
-        tmem_ld_32x32b_x32(lane_addr + ACC_COL + 128 + half * 64, v[2]);
-        tmem_ld_32x32b_x32(lane_addr + ACC_COL + 128 + half * 64 + 32, v[3]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 128 + 32 * i, v[i]);
-      }
-      tmem_ld_wait();
+      epilogue_load(p, tmem, q, half, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.acc_empty);
-
-      const int row = mt * BM + 32 * q + lane;
-      if (row >= p.M) {
-        // padding rows of an NVFP4 output: their scale words are written as zero
-        if (p.out_kind == OUT_NVFP4) {
-          const int span = p.mode == MODE_SILU_MUL ? 64 : 128;
-          const int cbeg = p.mode == MODE_SILU_MUL ? nt * 128 + half * 64 : nt * BN + half * 128;
-          for (int cg = cbeg; cg < cbeg + span && cg < p.Nout; cg += 64)
-            *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, cg / 64, p.out_kb_atoms)) = 0u;
-        }
-        continue;
-      }
-      if (p.mode == MODE_SILU_MUL) {
-        // output columns [nt*128 + half*64, +64): gate = weight row n, up = row up_row0 + n
-        const int col0 = nt * 128 + half * 64;
-        const float ag = seg_alpha(c, p.nseg, col0);
-        const float au = seg_alpha(c, p.nseg, p.up_row0 + col0);
-        float h[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float g = ag * __uint_as_float(v[i >> 5][i & 31]);
-          const float u = au * __uint_as_float(v[2 + (i >> 5)][i & 31]);
-          h[i] = (g / (1.0f + expf(-g))) * u;
-        }
-        if (p.out_kind == OUT_NVFP4) {
-          store64_nvfp4(p, row, col0, h, gs_out);
-        } else {
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            float y[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) y[i] = h[16 * b + i];
-            store16(p, row, col0 + 16 * b, y);
-          }
-        }
-      } else {
-        const int col0 = nt * BN + half * 128;
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {  // two 64-column groups
-          const int cg = col0 + 64 * hb;
-          if (cg >= p.Nout) break;
-          float y[64];
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const float a = seg_alpha(c, p.nseg, cg + 16 * b);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) y[16 * b + i] = a * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
-          }
-          if (p.mode == MODE_GDN) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-              const int n = cg + i;
-              if (n >= p.beta_begin && n < p.beta_begin + p.n_heads) {
-                const float bt = sigmoid_f(y[i]);
-                y[i] = bt;
-                if (p.beta_out) p.beta_out[(int64_t)row * p.n_heads + (n - p.beta_begin)] = bt;
-              } else if (n >= p.alpha_begin && n < p.alpha_begin + p.n_heads) {
-                const int hh = n - p.alpha_begin;
-                const float g = -expf(__ldg(p.A_log + hh)) * softplus_f(y[i] + __ldg(p.dt_bias + hh));
-                y[i] = g;
-                if (p.g_out) p.g_out[(int64_t)row * p.n_heads + hh] = g;
-              }
-            }
-          }
-          if (p.out_kind == OUT_NVFP4) {
-            store64_nvfp4(p, row, cg, y, gs_out);
-          } else {
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-              if (cg + 16 * b < p.Nout) {
-                float yy[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) yy[i] = y[16 * b + i];
-                store16(p, row, cg + 16 * b, yy);
-              }
-            }
-          }
-        }
-      }
+      epilogue_row(p, c, v, mt * BM + 32 * q + lane, nt, half, gs_out);
     }
   }
 
@@ -412,6 +543,145 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ============================================================ 2-CTA kernel
+// Bytes one stage brings into ONE CTA (A rows, its B half, SFA, both SFB halves).
+constexpr uint32_t STAGE2_TX = A_BYTES + B_HALF_BYTES + SFA_BYTES + SFB_BYTES;
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                 const __grid_constant__ Params p) {
+  using P = Plan2;
+  constexpr int STAGES = P::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl<STAGES> &c = *reinterpret_cast<Ctrl<STAGES> *>(smem);
+  uint8_t *sA = smem + P::A_OFF;
+  uint8_t *sB = smem + P::B_OFF;
+  uint8_t *sSFA = smem + P::SFA_OFF;
+  uint8_t *sSFB = smem + P::SFB_OFF;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs and scale copies; 1: its peer
+  const int cid = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    init_barriers(c, 2 * NUM_EPI_WARPS);
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmSFA);
+    prefetch_tensormap(&tmSFB);
+  }
+  load_segments(p, c);
+  if (warp == 1) {
+    tmem_alloc_cg2(&c.tmem_base, TMEM_COLS);
+    tmem_relinquish_cg2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before either signals the other
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  const int num_tiles = p.m_tiles * p.n_tiles;
+  const int my_tiles = num_tiles > cid ? (num_tiles - 1 - cid) / nclusters + 1 : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;  // per-stage bit masks (rank 0 only)
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
+        int mt, nt, rb0, rb1;
+        tile_coords(p, tile, mt, nt);
+        b_rows(p, nt, rb0, rb1);
+        const int a_row = mt * (2 * BM) + (int)rank * BM;
+        const int b_row = rank == 0 ? rb0 : rb1;
+        for (int kt = 0; kt < p.k_tiles; ++kt) {
+          if (!mbar_wait(&c.empty[stage], phase ^ 1)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&c.full[stage], 2 * STAGE2_TX);
+          const uint32_t bar = mapa_shared(smem_u32(&c.full[stage]), 0);
+          const int kx = kt * (BK / 2);
+          const int ksf = kt * (SFA_BYTES / 8);  // scale tensor maps count 8-byte elements
+          tma_load_2d_cg2(sA + stage * A_BYTES, &tmA, bar, kx, a_row);
+          tma_load_2d_cg2(sB + stage * P::B_BYTES, &tmB, bar, kx, b_row);
+          tma_load_2d_cg2(sSFA + stage * SFA_BYTES, &tmSFA, bar, ksf, a_row >> 7);
+          tma_load_2d_cg2(sSFB + stage * SFB_BYTES, &tmSFB, bar, ksf, rb0 >> 7);
+          tma_load_2d_cg2(sSFB + stage * SFB_BYTES + SFB_HALF_BYTES, &tmSFB, bar, ksf, rb1 >> 7);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // the even CTA's barriers count both CTAs' bytes: let them all land before exit
+      if (rank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&c.full[s], (armed_phase >> s) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = make_idesc(2 * BM, BN);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
+        if (!mbar_wait_cluster(&c.acc_empty, acc_phase ^ 1)) break;
+        acc_phase ^= 1;
+        tc_fence_after();
+        for (int kt = 0; kt < p.k_tiles; ++kt) {
+          if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t a_desc = sdesc_sw128_kmajor(smem_u32(sA + stage * A_BYTES));
+          const uint64_t b_desc = sdesc_sw128_kmajor(smem_u32(sB + stage * P::B_BYTES));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            mma_nvfp4_cg2(tmem + ACC_COL, a_desc + 2 * j, b_desc + 2 * j, idesc, tmem + sfa_col(stage) + 4 * j,
+                          tmem + sfb_col(stage) + 8 * j, (kt | j) != 0);
+          }
+          tc_commit_mc_cg2(&c.empty[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (ok) tc_commit_mc_cg2(&c.acc_full, 0x3);
+      }
+      // wait for every tcgen05 operation this thread issued
+      tc_commit_cg2(&c.drain);
+      mbar_wait(&c.drain, 0);
+    }
+  } else if (warp == COPY_WARP) {
+    if (lane == 0 && rank == 0) copy_scales<STAGES, true>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles);
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    uint32_t acc_phase = 0;
+    const float gs_out = p.out_kind == OUT_NVFP4 ? __ldg(p.gs_out) : 1.0f;
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(&c.acc_empty), 0);
+    for (int tile = cid; tile < num_tiles; tile += nclusters) {
+      int mt, nt;
+      tile_coords(p, tile, mt, nt);
+      if (!mbar_wait(&c.acc_full, acc_phase)) break;
+      acc_phase ^= 1;
+      tc_fence_after();
+      uint32_t v[4][32];
+      epilogue_load(p, tmem, q, half, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0);
+      epilogue_row(p, c, v, mt * (2 * BM) + (int)rank * BM + 32 * q + lane, nt, half, gs_out);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the other may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_cg2(tmem, TMEM_COLS);
 }
 
 }  // namespace gemm

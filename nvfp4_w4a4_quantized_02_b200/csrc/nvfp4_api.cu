@@ -23,6 +23,7 @@ struct DeviceInfo {
   int sms = 0;
   bool attrs = false;
   int quant_ctas_per_sm = 1;
+  int gemm2_clusters = 1;  // co-resident 2-CTA clusters of gemm2_kernel
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -48,11 +49,31 @@ nvfp4_status_t current_device(DeviceInfo **info) {
   }
   if (!d.ok) return NVFP4_ERR_UNSUPPORTED_DEVICE;
   if (!d.attrs) {
-    if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
+    if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::Plan1::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::Plan2::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
             cudaSuccess ||
         cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes) !=
             cudaSuccess)
       return NVFP4_ERR_CUDA;
+    {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * d.sms, 1, 1);
+      cfg.blockDim = dim3(gemm::NUM_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = gemm::Plan2::BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm::gemm2_kernel, &cfg) != cudaSuccess) return NVFP4_ERR_CUDA;
+      d.gemm2_clusters = clusters < 1 ? 1 : clusters;
+    }
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel, kQThreads, kQSmemBytes) != cudaSuccess)
       return NVFP4_ERR_CUDA;
@@ -107,6 +128,22 @@ bool make_bf16_map(CUtensorMap *m, const void *x, int64_t rows, int64_t cols, in
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor map of a swizzled scale buffer of a [rows x K] operand, viewed as 8-byte
+// elements: one row per 128-row group (K/64 atoms of 512 bytes), boxes of 256
+// elements = the 4 atoms (2 KB) of one 256-wide K tile of one group.
+bool make_scales_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_t K) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int64_t groups = (rows + 127) / 128;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 64 * 64), static_cast<cuuint64_t>(groups)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 64 * 512)};
+  cuuint32_t box[2] = {256, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -253,8 +290,11 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;
 
-  CUtensorMap tmA, tmB;
+  const bool pair = M > BM;  // 2-CTA tiles of 256 rows; one CTA per tile for M <= 128
+  CUtensorMap tmA, tmB, tmSFA, tmSFB;
   if (!make_codes_map(&tmA, A->codes, M, K) || !make_codes_map(&tmB, W->codes, N, K)) return NVFP4_ERR_CUDA;
+  if (pair && (!make_scales_map(&tmSFA, A->scales, M, K) || !make_scales_map(&tmSFB, W->scales, N, K)))
+    return NVFP4_ERR_CUDA;
 
   Params p{};
   p.M = static_cast<int>(M);
@@ -263,14 +303,14 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   p.Nout = static_cast<int>(Nout);
   p.mode = epilogue;
   p.out_kind = out_kind;
-  p.m_tiles = static_cast<int>((M + BM - 1) / BM);
+  const int64_t tile_m = pair ? 2 * BM : BM;
+  p.m_tiles = static_cast<int>((M + tile_m - 1) / tile_m);
   p.n_tiles = epilogue == NVFP4_EPI_SILU_MUL ? static_cast<int>(Nout / 128) : static_cast<int>((N + BN - 1) / BN);
   p.k_tiles = static_cast<int>(K / BK);
   p.up_row0 = static_cast<int>(Nout);
   p.kb_atoms = K / 64;
   p.sfa = A->scales;
   p.sfb = W->scales;
-  p.w_rows_pad = static_cast<int>((N + 127) / 128 * 128);
   p.gs_a = gs_a;
   p.nseg = nseg;
   for (int i = 0; i < nseg; ++i) {
@@ -298,8 +338,26 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   }
   const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles;
   if (tiles > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
-  gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(tmA, tmB, p);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!pair) {
+    const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
+    gemm_kernel<<<grid, NUM_THREADS, Plan1::BYTES, st>>>(tmA, tmB, p);
+    return launch_status();
+  }
+  const int64_t clusters = tiles < dev->gemm2_clusters ? tiles : dev->gemm2_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Plan2::BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm2_kernel, tmA, tmB, tmSFA, tmSFB, p) != cudaSuccess) return NVFP4_ERR_CUDA;
   return launch_status();
 }
 

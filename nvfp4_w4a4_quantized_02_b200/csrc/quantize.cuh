@@ -167,10 +167,6 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
     uint4 v[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) v[q] = *reinterpret_cast<const uint4 *>(rowp + (((4 * h + q) ^ (rho & 7)) << 4));
-    if (__syncthreads_or(!ok)) break;  // stage s fully read (or a copy never landed)
-    done = i + 1;
-    if (tid == 0 && issued < my_n) issue(issued++);
-
     uint32_t code[4];
     uint32_t sf2 = 0;
 #pragma unroll
@@ -191,6 +187,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
       code[2 * b + 1] = encode8(x + 8, inv);
       sf2 |= sf << (8 * b);
     }
+    // Stage s is refilled by the TMA (async proxy) once every thread is past this
+    // point: the proxy fence orders this thread's shared loads of the stage before
+    // that write, so the copy cannot overtake a load still in flight.
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (__syncthreads_or(!ok)) break;  // (or a copy never landed)
+    done = i + 1;
+    if (tid == 0 && issued < my_n) issue(issued++);
 
     const int64_t dest = rt * kQTileRows + rho;
     const bool own = dest >= a.row_offset && dest < a.own_end;

@@ -60,10 +60,16 @@ def test_exact_power_of_two_scales_pin_scale_layout(nv):
     assert np.array_equal(got, ref), f"{np.sum(got != ref)} mismatches"
 
 
-def test_single_nonzero_probes(nv):
-    """One non-zero code / scale at a time lands in exactly one output element."""
-    M, N, K = 128, 256, 256
-    for (m, n, k) in [(0, 0, 0), (5, 7, 1), (37, 130, 77), (127, 255, 255), (64, 200, 128), (96, 31, 200)]:
+@pytest.mark.parametrize("M", [128, 256])
+def test_single_nonzero_probes(nv, M):
+    """One non-zero code / scale at a time lands in exactly one output element.
+    M = 128 runs the one-CTA kernel, M = 256 the CTA-pair kernel (rows 128..255 and
+    B rows 128..255 come from the second CTA of the pair)."""
+    N, K = 256, 256
+    probes = [(0, 0, 0), (5, 7, 1), (37, 130, 77), (127, 255, 255), (64, 200, 128), (96, 31, 200)]
+    if M > 128:
+        probes += [(128, 0, 0), (200, 129, 63), (255, 255, 255), (131, 3, 250)]
+    for (m, n, k) in probes:
         ca = np.zeros((M, K), np.uint8)
         cw = np.zeros((N, K), np.uint8)
         ca[m, k] = 7      # 6.0
@@ -172,11 +178,14 @@ def test_gdn_gates_epilogue(nv):
         assert not bad.any(), (np.argwhere(bad)[:4], got[bad][:4], ref[bad][:4])
 
 
-def test_silu_mul_epilogue_and_requant(nv):
+@pytest.mark.parametrize("M", [256, 300])
+def test_silu_mul_epilogue_and_requant(nv, M):
     """MLP gate|up with SiLU*mul: BF16 output vs oracle, and the fused NVFP4
-    re-quantisation equal (bit for bit) to BF16 output + the standalone quantiser."""
+    re-quantisation equal (bit for bit) to BF16 output + the standalone quantiser.
+    M = 300: the last CTA pair covers rows 256..511, of which 300..383 are scale
+    padding (written as zero) and 384..511 lie outside the output."""
     import torch
-    M, K, Nh = 256, 512, 256
+    K, Nh = 512, 256
     ws = synth.segmented_weights([("gate", Nh), ("up", Nh)], K, seed=31, multipliers={"gate": 1, "up": 2})
     xb = synth.student_t_activations(M, K, seed=30)
     ca, sa, gsa = oracle_quant(xb)
@@ -194,7 +203,9 @@ def test_silu_mul_epilogue_and_requant(nv):
     assert_gemm_close(h16, h_ref)
     # fused requant == unfused BF16 output quantised by the standalone kernel
     gs_h = nv.global_scale(h16)
-    hq = nv.linear(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=gs_h)
+    out_scales = torch.full((nv.scale_bytes(M, Nh),), 0xAB, dtype=torch.uint8, device="cuda")
+    hq = nv.linear(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=gs_h,
+                   out_scales=out_scales)
     hq2 = nv.quantize(h16, gs_h)
     _sync()
     assert torch.equal(hq.codes, hq2.codes)
