@@ -20,7 +20,7 @@
 //   both CTAs.  Each TMA load is a plain load of one CTA's own tile from this GPU's
 //   memory.
 //
-// Roles (one persistent CTA per SM, 352 threads):
+// Roles (one persistent CTA per SM, 384 threads):
 //   warp 0      TMA producer: code tiles (128-byte swizzle) and scale tiles (already
 //               in the MMA's 128 x 4 atom layout) into a shared-memory ring.
 //   warp 1      MMA issuer: 4 block-scaled MMAs (K = 64 each) per stage into the
@@ -28,12 +28,14 @@
 //   warps 2..9  epilogue: tcgen05.ld the 128 x 256 FP32 accumulator (each warp a
 //               32-lane quadrant x 128 columns) into registers, hand TMEM back to the
 //               MMA warp at once, then scale / activate / store from registers.
-//   warp 10     scale copier: per stage, 12 tcgen05.cp of the A and B scale atoms
-//               into that stage's TMEM scale columns, then tcgen05.commit to the
-//               MMA issuer.  Issued from their own thread, the copies of stage s+1
-//               overlap the MMAs of stage s; issued in line with the MMAs they ran
-//               in series with them and cost ~60 cycles each (measured: gate|up
-//               GEMM of the MLP block 3.26 ms -> 2.76 ms with the 1-CTA kernel).
+//   warps 10,11 scale copiers: per stage, 12 tcgen05.cp of the A and B scale atoms
+//               (6 per warp) into that stage's TMEM scale columns, then
+//               tcgen05.commit to the MMA issuer.  Issued from their own threads, the
+//               copies of stage s+1 overlap the MMAs of stage s; issued in line with
+//               the MMAs they ran in series with them and cost ~60 cycles each
+//               (measured on the MLP block's gate|up GEMM, 1-CTA kernel: 3.26 ms in
+//               line, 2.76 ms with one copier; CTA-pair kernel: 2.55 ms with one
+//               copier, 2.50 ms with two).
 // Output tiles are visited in groups of 16 M-tiles so that concurrently running
 // CTAs share A and W tiles in L2.
 #pragma once
@@ -53,8 +55,9 @@ constexpr int SFA_BYTES = 4 * SF_ATOM;   // 4 MMA k-steps
 constexpr int SFB_HALF_BYTES = 4 * SF_ATOM;
 constexpr int SFB_BYTES = 2 * SFB_HALF_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int COPY_WARP = 2 + NUM_EPI_WARPS;
-constexpr int NUM_THREADS = 32 * (COPY_WARP + 1);
+constexpr int COPY_WARP = 2 + NUM_EPI_WARPS;  // first of the scale-copy warps
+constexpr int NUM_COPY_WARPS = 2;  // copy_scales splits a stage's 12 atoms in two halves
+constexpr int NUM_THREADS = 32 * (COPY_WARP + NUM_COPY_WARPS);
 constexpr int GROUP_M = 16;
 
 // TMEM columns (allocation of 512 = the whole TMEM of the SM): the 256-column FP32
@@ -132,8 +135,8 @@ struct Ctrl {
   int seg_end[16];
   float seg_alpha[16];
   float inv_out[128];  // NVFP4 output: gs_out / e4m3(sf) for sf = 0..127 (0 for 0 and NaN)
-  uint64_t sf_ready[STAGES];  // the stage's scales are in TMEM (tcgen05.commit of the copier)
-  uint64_t sf_drain;
+  uint64_t sf_ready[STAGES];  // the stage's scales are in TMEM (tcgen05.commit of both copiers)
+  uint64_t sf_drain[NUM_COPY_WARPS];
 };
 static_assert(sizeof(Ctrl<6>) <= 1024, "control block too large");
 
@@ -352,34 +355,43 @@ __device__ __forceinline__ void load_segments(const Params &p, Ctrl<STAGES> &c) 
   }
 }
 
-// Scale copier (one thread): for each stage of the CTA's run, once the stage's
-// bytes landed, copy its scale atoms into the stage's TMEM scale set and commit to
-// sf_ready[stage].  Set s is rewritten only after full[s] completed again, i.e.
-// after the producer refilled stage s, which waited for the MMAs that read set s.
+// Scale copier `part` (one thread of warp COPY_WARP + part): for each stage of the
+// CTA's run, once the stage's bytes landed, copy half of its 12 scale atoms into the
+// stage's TMEM scale set and commit to sf_ready[stage] (which waits for both
+// copiers).  Part 0: A's 4 k-steps and B's first half for k-steps 0, 1; part 1: B's
+// first half for k-steps 2, 3 and B's second half.  Set s is rewritten only after
+// full[s] completed again, i.e. after the producer refilled stage s, which waited
+// for the MMAs that read set s.
+template <bool kPair>
+__device__ __forceinline__ void cp_scale_atom(uint32_t taddr, uint32_t saddr) {
+  if constexpr (kPair) {  // each CTA's atom goes to its own TMEM (same addresses in both)
+    tc_cp_32x128b_x4_cg2(taddr, sdesc_plain_32x16B(saddr));
+  } else {
+    tc_cp_32x128b_x4(taddr, sdesc_plain_32x16B(saddr));
+  }
+}
+
 template <int STAGES, bool kPair>
 __device__ __forceinline__ void copy_scales(Ctrl<STAGES> &c, uint32_t tmem, const uint8_t *sSFA,
-                                            const uint8_t *sSFB, int total) {
+                                            const uint8_t *sSFB, int total, int part) {
   int stage = 0;
   uint32_t phase = 0;
   for (int g = 0; g < total; ++g) {
     if (!mbar_wait(&c.full[stage], phase)) break;
     tc_fence_after();
-    const uint32_t sfa_addr = smem_u32(sSFA + stage * SFA_BYTES);
-    const uint32_t sfb_addr = smem_u32(sSFB + stage * SFB_BYTES);
+    const uint32_t sfa = smem_u32(sSFA + stage * SFA_BYTES);
+    const uint32_t sfb = smem_u32(sSFB + stage * SFB_BYTES);
+    if (part == 0) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint64_t da = sdesc_plain_32x16B(sfa_addr + j * SF_ATOM);
-      const uint64_t db0 = sdesc_plain_32x16B(sfb_addr + j * SF_ATOM);
-      const uint64_t db1 = sdesc_plain_32x16B(sfb_addr + SFB_HALF_BYTES + j * SF_ATOM);
-      if constexpr (kPair) {  // each CTA's scales go to its own TMEM (same addresses in both)
-        tc_cp_32x128b_x4_cg2(tmem + sfa_col(stage) + 4 * j, da);
-        tc_cp_32x128b_x4_cg2(tmem + sfb_col(stage) + 8 * j, db0);
-        tc_cp_32x128b_x4_cg2(tmem + sfb_col(stage) + 8 * j + 4, db1);
-      } else {
-        tc_cp_32x128b_x4(tmem + sfa_col(stage) + 4 * j, da);
-        tc_cp_32x128b_x4(tmem + sfb_col(stage) + 8 * j, db0);
-        tc_cp_32x128b_x4(tmem + sfb_col(stage) + 8 * j + 4, db1);
-      }
+      for (int j = 0; j < 4; ++j) cp_scale_atom<kPair>(tmem + sfa_col(stage) + 4 * j, sfa + j * SF_ATOM);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) cp_scale_atom<kPair>(tmem + sfb_col(stage) + 8 * j, sfb + j * SF_ATOM);
+    } else {
+#pragma unroll
+      for (int j = 2; j < 4; ++j) cp_scale_atom<kPair>(tmem + sfb_col(stage) + 8 * j, sfb + j * SF_ATOM);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        cp_scale_atom<kPair>(tmem + sfb_col(stage) + 8 * j + 4, sfb + SFB_HALF_BYTES + j * SF_ATOM);
     }
     if constexpr (kPair) {
       tc_commit_cg2(&c.sf_ready[stage]);
@@ -389,12 +401,13 @@ __device__ __forceinline__ void copy_scales(Ctrl<STAGES> &c, uint32_t tmem, cons
     if (++stage == STAGES) { stage = 0; phase ^= 1; }
   }
   // wait for every copy this thread issued
+  uint64_t *drain = &c.sf_drain[part];
   if constexpr (kPair) {
-    tc_commit_cg2(&c.sf_drain);
+    tc_commit_cg2(drain);
   } else {
-    tc_commit(&c.sf_drain);
+    tc_commit(drain);
   }
-  mbar_wait(&c.sf_drain, 0);
+  mbar_wait(drain, 0);
 }
 
 template <int STAGES>
@@ -402,12 +415,12 @@ __device__ __forceinline__ void init_barriers(Ctrl<STAGES> &c, uint32_t acc_empt
   for (int s = 0; s < STAGES; ++s) {
     mbar_init(&c.full[s], 1);
     mbar_init(&c.empty[s], 1);
-    mbar_init(&c.sf_ready[s], 1);
+    mbar_init(&c.sf_ready[s], NUM_COPY_WARPS);
   }
   mbar_init(&c.acc_full, 1);
   mbar_init(&c.acc_empty, acc_empty_count);
   mbar_init(&c.drain, 1);
-  mbar_init(&c.sf_drain, 1);
+  for (int i = 0; i < NUM_COPY_WARPS; ++i) mbar_init(&c.sf_drain[i], 1);
   fence_barrier_init();
 }
 
@@ -516,8 +529,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(&c.drain);
       mbar_wait(&c.drain, 0);
     }
-  } else if (warp == COPY_WARP) {
-    if (lane == 0) copy_scales<STAGES, false>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles);
+  } else if (warp >= COPY_WARP) {
+    if (lane == 0) copy_scales<STAGES, false>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles, warp - COPY_WARP);
   } else {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
@@ -653,8 +666,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit_cg2(&c.drain);
       mbar_wait(&c.drain, 0);
     }
-  } else if (warp == COPY_WARP) {
-    if (lane == 0 && rank == 0) copy_scales<STAGES, true>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles);
+  } else if (warp >= COPY_WARP) {
+    if (lane == 0 && rank == 0)
+      copy_scales<STAGES, true>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles, warp - COPY_WARP);
   } else {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;
