@@ -121,6 +121,15 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(value: float, device) -> float:
+    """Largest ``value`` over the ranks of the default process group (the job's time
+    is the slowest rank's)."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def sources_hash(files):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "nvfp4_w4a4_quantized_02_b200", "csrc")
@@ -732,9 +741,7 @@ def run_ours(args, ws, rank):
     else:
         elapsed_ms = start.elapsed_time(stop)
     if ws > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+        elapsed_ms = max_over_ranks(elapsed_ms, "cuda")
         torch.distributed.barrier()
 
     ksum = tm.summary()
