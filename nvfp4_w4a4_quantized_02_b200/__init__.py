@@ -14,6 +14,7 @@ from typing import Optional, Sequence
 
 __all__ = [
     "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
+    "linear_splitk", "splitk_default", "splitk_workspace_bytes",
     "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
 ]
 
@@ -50,7 +51,8 @@ class NVFP4Error(RuntimeError):
 
 _LIB = None
 SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
-           "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_get_device_status")
+           "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
+           "nvfp4_splitk_default", "nvfp4_get_device_status")
 
 
 def lib():
@@ -77,6 +79,15 @@ def lib():
     L.nvfp4_linear.argtypes = [ctypes.POINTER(Operand), _c_vp, ctypes.POINTER(Operand),
                                ctypes.POINTER(Segment), ctypes.c_int, ctypes.c_int,
                                ctypes.POINTER(EpilogueParams), _c_vp, ctypes.c_int, _c_i64, _c_vp]
+    L.nvfp4_linear_splitk.restype = ctypes.c_int
+    L.nvfp4_linear_splitk.argtypes = [ctypes.POINTER(Operand), _c_vp, ctypes.POINTER(Operand),
+                                      ctypes.POINTER(Segment), ctypes.c_int, ctypes.c_int,
+                                      ctypes.POINTER(EpilogueParams), _c_vp, ctypes.c_int, _c_i64,
+                                      ctypes.c_int, _c_vp, ctypes.c_size_t, _c_vp]
+    L.nvfp4_splitk_workspace_bytes.restype = ctypes.c_size_t
+    L.nvfp4_splitk_workspace_bytes.argtypes = [_c_i64, _c_i64, ctypes.c_int]
+    L.nvfp4_splitk_default.restype = ctypes.c_int
+    L.nvfp4_splitk_default.argtypes = [_c_i64, _c_i64, _c_i64]
     L.nvfp4_get_device_status.restype = ctypes.c_int
     L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     _LIB = L
@@ -175,18 +186,9 @@ def quantize_fused(parts, gs_list=None, stream=None):
     return NVFP4Tensor(codes, scales, segs[0][2], total, cols), segs
 
 
-def linear(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None, epilogue: str = "none",
-           out_dtype: str = "bf16", out=None, ldo: Optional[int] = None, gates: Optional[dict] = None,
-           gs_out=None, out_scales=None, stream=None):
-    """Fused W4A4 linear ``epilogue(A @ W^T / (gs_a * gs_w[seg]))``.
-
-    segments: list of ``(n_begin, n_end, gs_w_tensor)``; default one segment with ``w.gs``.
-    gates (gdn_gates): dict with beta_begin, alpha_begin, n_heads, A_log, dt_bias
-    [, beta_out, g_out] (float32 device tensors).
-    out_dtype "nvfp4" returns an NVFP4Tensor quantised with ``gs_out``.
-    """
+def _linear_args(a, w, segments, epilogue, out_dtype, out, ldo, gates, gs_out, out_scales):
+    """Marshal the arguments shared by nvfp4_linear and nvfp4_linear_splitk."""
     import torch
-    L = lib()
     M, K = a.rows, a.cols
     N = w.rows
     if segments is None:
@@ -201,7 +203,6 @@ def linear(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None, 
         ep.beta_begin, ep.alpha_begin, ep.n_heads = int(g["beta_begin"]), int(g["alpha_begin"]), int(g["n_heads"])
         ep.A_log, ep.dt_bias = _ptr(g["A_log"]), _ptr(g["dt_bias"])
         ep.beta_out, ep.g_out = _ptr(g.get("beta_out")), _ptr(g.get("g_out"))
-    result = None
     if out_dtype == "nvfp4":
         if gs_out is None:
             raise ValueError("nvfp4 output needs gs_out")
@@ -220,9 +221,54 @@ def linear(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None, 
         result = out
     A = Operand(a.codes.data_ptr(), a.scales.data_ptr(), M, K)
     W = Operand(w.codes.data_ptr(), w.scales.data_ptr(), N, w.cols)
-    _check(L.nvfp4_linear(ctypes.byref(A), _c_vp(a.gs.data_ptr()), ctypes.byref(W), segs, len(segments),
-                          EPILOGUES[epilogue], ctypes.byref(ep), _c_vp(out.data_ptr()), OUT_KINDS[out_dtype],
-                          int(ldo), _stream(stream)), "nvfp4_linear")
+    args = (ctypes.byref(A), _c_vp(a.gs.data_ptr()), ctypes.byref(W), segs, len(segments),
+            EPILOGUES[epilogue], ctypes.byref(ep), _c_vp(out.data_ptr()), OUT_KINDS[out_dtype], int(ldo))
+    keep = (A, W, segs, ep)  # keep the ctypes structures alive across the call
+    return args, result, keep
+
+
+def linear(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None, epilogue: str = "none",
+           out_dtype: str = "bf16", out=None, ldo: Optional[int] = None, gates: Optional[dict] = None,
+           gs_out=None, out_scales=None, stream=None):
+    """Fused W4A4 linear ``epilogue(A @ W^T / (gs_a * gs_w[seg]))``.
+
+    segments: list of ``(n_begin, n_end, gs_w_tensor)``; default one segment with ``w.gs``.
+    gates (gdn_gates): dict with beta_begin, alpha_begin, n_heads, A_log, dt_bias
+    [, beta_out, g_out] (float32 device tensors).
+    out_dtype "nvfp4" returns an NVFP4Tensor quantised with ``gs_out``.
+    """
+    args, result, _keep = _linear_args(a, w, segments, epilogue, out_dtype, out, ldo, gates, gs_out, out_scales)
+    _check(lib().nvfp4_linear(*args, _stream(stream)), "nvfp4_linear")
+    return result
+
+
+def splitk_default(M: int, N: int, K: int) -> int:
+    return int(lib().nvfp4_splitk_default(M, N, K))
+
+
+def splitk_workspace_bytes(M: int, N: int, split_k: int) -> int:
+    return int(lib().nvfp4_splitk_workspace_bytes(M, N, split_k))
+
+
+def linear_splitk(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None, epilogue: str = "none",
+                  out_dtype: str = "bf16", out=None, ldo: Optional[int] = None, gates: Optional[dict] = None,
+                  gs_out=None, out_scales=None, split_k: Optional[int] = None, workspace=None, stream=None):
+    """``linear`` with K split over ``split_k`` units per output tile (decode regime).
+
+    ``workspace``: a CUDA tensor of at least ``splitk_workspace_bytes(M, N, split_k)``
+    bytes (allocated here when None).  ``split_k`` None: the library's choice.
+    """
+    import torch
+    M, N, K = a.rows, w.rows, a.cols
+    if split_k is None:
+        split_k = splitk_default(M, N, K)
+    need = splitk_workspace_bytes(M, N, split_k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=a.codes.device)
+    args, result, _keep = _linear_args(a, w, segments, epilogue, out_dtype, out, ldo, gates, gs_out, out_scales)
+    _check(lib().nvfp4_linear_splitk(*args, int(split_k), _c_vp(workspace.data_ptr()),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "nvfp4_linear_splitk")
     return result
 
 

@@ -103,7 +103,10 @@ struct Segment {
 struct Params {
   int M, N, K, Nout;
   int mode, out_kind;
+  int tile_mode;                  // how B tiles are formed and read back: mode, or MODE_NONE for split-K
   int m_tiles, n_tiles, k_tiles;  // m_tiles counts tiles of BM * (CTAs per tile) rows
+  int splits, kt_per_split;       // split-K: K tiles [s * kt_per_split, ...) form split s (1 split: whole K)
+  float *partial;                 // split-K: FP32 partial sums [splits][M][N]; null otherwise
   int up_row0;              // SILU_MUL: first weight row of the `up` half
   int64_t kb_atoms;         // K / 64
   const uint8_t *sfa;       // swizzled scales of A
@@ -157,13 +160,21 @@ __device__ __forceinline__ void tile_coords(const Params &p, int tile, int &mt, 
 
 // First weight rows of the two 128-row halves of the B tile of N-tile nt.
 __device__ __forceinline__ void b_rows(const Params &p, int nt, int &rb0, int &rb1) {
-  if (p.mode == MODE_SILU_MUL) {
+  if (p.tile_mode == MODE_SILU_MUL) {
     rb0 = nt * 128;
     rb1 = p.up_row0 + nt * 128;
   } else {
     rb0 = nt * BN;
     rb1 = nt * BN + 128;
   }
+}
+
+// Work unit u of a launch: output tile u / splits, K tiles [k0, k1) of split u % splits.
+__device__ __forceinline__ void unit_coords(const Params &p, int u, int &tile, int &split, int &k0, int &k1) {
+  tile = u / p.splits;
+  split = u - tile * p.splits;
+  k0 = split * p.kt_per_split;
+  k1 = min(p.k_tiles, k0 + p.kt_per_split);
 }
 
 template <int STAGES>
@@ -175,6 +186,7 @@ __device__ __forceinline__ float seg_alpha(const Ctrl<STAGES> &c, int nseg, int 
 }
 
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+__device__ __forceinline__ float silu_mul_f(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x))); }
 
 // Store 16 consecutive output values of one row.
@@ -248,7 +260,7 @@ __device__ __noinline__ void gdn_gates64(const Params &p, int row, int cg, float
 __device__ __forceinline__ void epilogue_load(const Params &p, uint32_t tmem, int q, int half,
                                               uint32_t (&v)[4][32]) {
   const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-  if (p.mode == MODE_SILU_MUL) {
+  if (p.tile_mode == MODE_SILU_MUL) {
     tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 64, v[0]);
     tmem_ld_32x32b_x32(lane_addr + ACC_COL + half * 64 + 32, v[1]);
     tmem_ld_32x32b_x32(lane_addr + ACC_COL + 128 + half * 64, v[2]);
@@ -280,14 +292,17 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
   if (p.mode == MODE_SILU_MUL) {
     // output columns [nt*128 + half*64, +64): gate = weight row n, up = row up_row0 + n
     const int col0 = nt * 128 + half * 64;
-    const float ag = seg_alpha(c, p.nseg, col0);
-    const float au = seg_alpha(c, p.nseg, p.up_row0 + col0);
     float h[64];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float g = ag * __uint_as_float(v[i >> 5][i & 31]);
-      const float u = au * __uint_as_float(v[2 + (i >> 5)][i & 31]);
-      h[i] = __fdividef(g, 1.0f + __expf(-g)) * u;  // SiLU(g) * u
+    for (int b = 0; b < 4; ++b) {
+      const float ag = seg_alpha(c, p.nseg, col0 + 16 * b);
+      const float au = seg_alpha(c, p.nseg, p.up_row0 + col0 + 16 * b);
+#pragma unroll
+      for (int i = 16 * b; i < 16 * b + 16; ++i) {
+        const float g = ag * __uint_as_float(v[i >> 5][i & 31]);
+        const float u = au * __uint_as_float(v[2 + (i >> 5)][i & 31]);
+        h[i] = silu_mul_f(g, u);
+      }
     }
     if (p.out_kind == OUT_NVFP4) {
       store64_nvfp4(p, c.inv_out, row, col0, h, gs_out);
@@ -335,6 +350,23 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
           store16(p, row, cg + 16 * b, yy);
         }
       }
+    }
+  }
+}
+
+// Split-K: the raw FP32 sums of 128 consecutive columns of one row, for split `split`.
+__device__ __forceinline__ void store_partial(const Params &p, const uint32_t (&v)[4][32], int split, int row,
+                                              int col0) {
+  if (row >= p.M) return;
+  float *dst = p.partial + ((int64_t)split * p.M + row) * p.N + col0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4) {
+      if (col0 + 32 * i + 4 * c4 < p.N)  // N % 16 == 0: a vector is all in or all out
+        *reinterpret_cast<float4 *>(dst + 32 * i + 4 * c4) =
+            make_float4(__uint_as_float(v[i][4 * c4]), __uint_as_float(v[i][4 * c4 + 1]),
+                        __uint_as_float(v[i][4 * c4 + 2]), __uint_as_float(v[i][4 * c4 + 3]));
     }
   }
 }
@@ -455,8 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
-  const int num_tiles = p.m_tiles * p.n_tiles;
-  const int my_tiles = num_tiles > (int)blockIdx.x ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int num_units = p.m_tiles * p.n_tiles * p.splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -465,8 +496,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_phase = 0;  // per-stage bit masks
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mt, nt, rb0, rb1;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        int tile, split, k0, k1, mt, nt, rb0, rb1;
+        unit_coords(p, u, tile, split, k0, k1);
         tile_coords(p, tile, mt, nt);
         b_rows(p, nt, rb0, rb1);
         const bool second = rb1 < p.N;  // any valid row in the second half
@@ -475,7 +507,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint8_t *sfa_src = p.sfa + ((int64_t)mt * p.kb_atoms) * SF_ATOM;
         const uint8_t *sfb0_src = p.sfb + ((int64_t)(rb0 >> 7) * p.kb_atoms) * SF_ATOM;
         const uint8_t *sfb1_src = p.sfb + ((int64_t)(rb1 >> 7) * p.kb_atoms) * SF_ATOM;
-        for (int kt = 0; kt < p.k_tiles; ++kt) {
+        for (int kt = k0; kt < k1; ++kt) {
           if (!mbar_wait(&c.empty[stage], phase ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&c.full[stage], bytes);
           const int kx = kt * (BK / 2);
@@ -505,11 +537,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        int tile, split, k0, k1;
+        unit_coords(p, u, tile, split, k0, k1);
         if (!mbar_wait(&c.acc_empty, acc_phase ^ 1)) break;
         acc_phase ^= 1;
         tc_fence_after();
-        for (int kt = 0; kt < p.k_tiles; ++kt) {
+        for (int kt = k0; kt < k1; ++kt) {
           if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
           tc_fence_after();
           const uint64_t a_desc = sdesc_sw128_kmajor(smem_u32(sA + stage * A_BYTES));
@@ -518,7 +552,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int j = 0; j < 4; ++j) {
             // advance 64 FP4 = 32 bytes along K inside the swizzle atom (+2 in 16-byte units)
             mma_nvfp4(tmem + ACC_COL, a_desc + 2 * j, b_desc + 2 * j, idesc, tmem + sfa_col(stage) + 4 * j,
-                      tmem + sfb_col(stage) + 8 * j, (kt | j) != 0);
+                      tmem + sfb_col(stage) + 8 * j, (kt != k0) | (j != 0));
           }
           tc_commit(&c.empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -530,15 +564,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&c.drain, 0);
     }
   } else if (warp >= COPY_WARP) {
-    if (lane == 0) copy_scales<STAGES, false>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles, warp - COPY_WARP);
+    if (lane == 0) {
+      int total = 0;  // stages this CTA runs through
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        int tile, split, k0, k1;
+        unit_coords(p, u, tile, split, k0, k1);
+        total += k1 - k0;
+      }
+      copy_scales<STAGES, false>(c, tmem, sSFA, sSFB, total, warp - COPY_WARP);
+    }
   } else {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2; // which 128 of the 256 accumulator columns
     uint32_t acc_phase = 0;
     const float gs_out = p.out_kind == OUT_NVFP4 ? __ldg(p.gs_out) : 1.0f;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int mt, nt;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      int tile, split, k0, k1, mt, nt;
+      unit_coords(p, u, tile, split, k0, k1);
       tile_coords(p, tile, mt, nt);
       if (!mbar_wait(&c.acc_full, acc_phase)) break;
       acc_phase ^= 1;
@@ -548,7 +591,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.acc_empty);
-      epilogue_row(p, c, v, mt * BM + 32 * q + lane, nt, half, gs_out);
+      const int row = mt * BM + 32 * q + lane;
+      if (p.partial) {
+        store_partial(p, v, split, row, nt * BN + half * 128);
+      } else {
+        epilogue_row(p, c, v, row, nt, half, gs_out);
+      }
     }
   }
 
@@ -696,6 +744,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   cluster_sync();  // neither CTA leaves while the other may still signal it
   tc_fence_after();
   if (warp == 1) tmem_dealloc_cg2(tmem, TMEM_COLS);
+}
+
+// ======================================================= split-K epilogue
+// Sums the splits' partials and applies the epilogue of the linear: one thread per
+// 64 output columns of one row (one scale word of an NVFP4 output).  Rows past M up
+// to the next multiple of 128 only write zero scale words (NVFP4 output).
+constexpr int REDUCE_THREADS = 256;
+
+// 16 consecutive column sums (col % 16 == 0, col + 16 <= N).
+__device__ __forceinline__ void partial_sum16(const Params &p, int row, int col, float (&y)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = 0.0f;
+  for (int sp = 0; sp < p.splits; ++sp) {
+    const float4 *src = reinterpret_cast<const float4 *>(p.partial + ((int64_t)sp * p.M + row) * p.N + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = src[i];
+      y[4 * i] += v.x;
+      y[4 * i + 1] += v.y;
+      y[4 * i + 2] += v.z;
+      y[4 * i + 3] += v.w;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(REDUCE_THREADS) splitk_epilogue_kernel(const __grid_constant__ Params p) {
+  __shared__ Ctrl<1> c;  // segment alphas and the NVFP4 output table
+  load_segments(p, c);
+  __syncthreads();
+  const int groups = (p.Nout + 63) / 64;
+  const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (int64_t)(p.M + 127) / 128 * 128 : p.M;
+  const int64_t idx = (int64_t)blockIdx.x * REDUCE_THREADS + threadIdx.x;
+  if (idx >= rows_cover * groups) return;
+  const int row = static_cast<int>(idx / groups);
+  const int cg = static_cast<int>(idx - (int64_t)row * groups) * 64;
+  if (row >= p.M) {
+    *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, cg / 64, p.out_kb_atoms)) = 0u;
+    return;
+  }
+  float y[64];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int col = cg + 16 * b;
+    float t[16];
+    if (col >= p.Nout) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) t[i] = 0.0f;
+    } else if (p.mode == MODE_SILU_MUL) {
+      float u[16];
+      partial_sum16(p, row, col, t);
+      partial_sum16(p, row, p.up_row0 + col, u);
+      const float ag = seg_alpha(c, p.nseg, col);
+      const float au = seg_alpha(c, p.nseg, p.up_row0 + col);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) t[i] = silu_mul_f(ag * t[i], au * u[i]);
+    } else {
+      partial_sum16(p, row, col, t);
+      const float a = seg_alpha(c, p.nseg, col);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) t[i] *= a;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[16 * b + i] = t[i];
+  }
+  if (p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + 64 > p.beta_begin) ||
+                             (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin))) {
+    float t[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) t[i] = y[i];
+    gdn_gates64(p, row, cg, t);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) y[i] = t[i];
+  }
+  if (p.out_kind == OUT_NVFP4) {
+    store64_nvfp4(p, c.inv_out, row, cg, y, __ldg(p.gs_out));
+  } else {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      if (cg + 16 * b < p.Nout) {
+        float yy[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) yy[i] = y[16 * b + i];
+        store16(p, row, cg + 16 * b, yy);
+      }
+    }
+  }
 }
 
 }  // namespace gemm

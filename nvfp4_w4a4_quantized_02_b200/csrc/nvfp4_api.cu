@@ -153,6 +153,138 @@ inline nvfp4_status_t launch_status() {
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
+// Validates the arguments of a linear and fills everything of Params but the tiling.
+nvfp4_status_t prepare_linear(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
+                              const nvfp4_segment_t *segs, int nseg, int epilogue,
+                              const nvfp4_epilogue_params_t *ep, void *out, int out_kind, int64_t ldo,
+                              gemm::Params &p) {
+  using namespace gemm;
+  if (!A || !W || !gs_a || !segs || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!A->codes || !A->scales || !W->codes || !W->scales) return NVFP4_ERR_INVALID_ARG;
+  if (A->rows < 1 || W->rows < 1 || A->K < 1 || A->K != W->K) return NVFP4_ERR_INVALID_ARG;
+  if (epilogue < NVFP4_EPI_NONE || epilogue > NVFP4_EPI_GDN_GATES) return NVFP4_ERR_INVALID_ARG;
+  if (out_kind < NVFP4_OUT_BF16 || out_kind > NVFP4_OUT_NVFP4) return NVFP4_ERR_INVALID_ARG;
+  if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  const int64_t M = A->rows, N = W->rows, K = A->K;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (K % BK != 0 || N % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  // segments: sorted, disjoint, 16-aligned, covering [0, N)
+  int64_t expect = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (!segs[i].gs_w || !aligned(segs[i].gs_w, 4)) return NVFP4_ERR_INVALID_ARG;
+    if (segs[i].n_begin != expect || segs[i].n_end <= segs[i].n_begin) return NVFP4_ERR_INVALID_ARG;
+    if (segs[i].n_begin % 16 != 0 || segs[i].n_end % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    expect = segs[i].n_end;
+  }
+  if (expect != N) return NVFP4_ERR_INVALID_ARG;
+  int64_t Nout = N;
+  if (epilogue == NVFP4_EPI_SILU_MUL) {
+    if (N % (2 * 128) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    Nout = N / 2;
+  }
+  if (epilogue == NVFP4_EPI_GDN_GATES) {
+    if (!ep || !ep->A_log || !ep->dt_bias || ep->n_heads < 1) return NVFP4_ERR_INVALID_ARG;
+    const int64_t h = ep->n_heads;
+    if (ep->beta_begin < 0 || ep->beta_begin + h > N || ep->alpha_begin < 0 || ep->alpha_begin + h > N)
+      return NVFP4_ERR_INVALID_ARG;
+    if (ep->beta_begin < ep->alpha_begin + h && ep->alpha_begin < ep->beta_begin + h) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(ep->A_log, 4) || !aligned(ep->dt_bias, 4) || (ep->beta_out && !aligned(ep->beta_out, 4)) ||
+        (ep->g_out && !aligned(ep->g_out, 4)))
+      return NVFP4_ERR_MISALIGNED;
+  }
+  if (out_kind == NVFP4_OUT_NVFP4) {
+    if (!ep || !ep->gs_out || !ep->out_scales) return NVFP4_ERR_INVALID_ARG;
+    if (Nout % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(out, 16) || !aligned(ep->out_scales, 16) || !aligned(ep->gs_out, 4)) return NVFP4_ERR_MISALIGNED;
+  } else {
+    const int64_t elem = out_kind == NVFP4_OUT_BF16 ? 2 : 4;
+    if (ldo < Nout) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || (ldo * elem) % 16 != 0) return NVFP4_ERR_MISALIGNED;
+  }
+  if (!aligned(A->codes, 16) || !aligned(W->codes, 16) || !aligned(A->scales, 16) || !aligned(W->scales, 16) ||
+      !aligned(gs_a, 4))
+    return NVFP4_ERR_MISALIGNED;
+
+  p = Params{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.Nout = static_cast<int>(Nout);
+  p.mode = epilogue;
+  p.tile_mode = epilogue;
+  p.out_kind = out_kind;
+  p.k_tiles = static_cast<int>(K / BK);
+  p.splits = 1;
+  p.kt_per_split = p.k_tiles;
+  p.partial = nullptr;
+  p.up_row0 = static_cast<int>(Nout);
+  p.kb_atoms = K / 64;
+  p.sfa = A->scales;
+  p.sfb = W->scales;
+  p.gs_a = gs_a;
+  p.nseg = nseg;
+  for (int i = 0; i < nseg; ++i) {
+    p.seg[i].n_begin = static_cast<int>(segs[i].n_begin);
+    p.seg[i].n_end = static_cast<int>(segs[i].n_end);
+    p.seg[i].gs_w = segs[i].gs_w;
+  }
+  p.out = out;
+  p.ldo = ldo;
+  p.beta_begin = p.alpha_begin = -1;
+  p.n_heads = 0;
+  if (epilogue == NVFP4_EPI_GDN_GATES) {
+    p.beta_begin = static_cast<int>(ep->beta_begin);
+    p.alpha_begin = static_cast<int>(ep->alpha_begin);
+    p.n_heads = static_cast<int>(ep->n_heads);
+    p.A_log = ep->A_log;
+    p.dt_bias = ep->dt_bias;
+    p.beta_out = ep->beta_out;
+    p.g_out = ep->g_out;
+  }
+  if (out_kind == NVFP4_OUT_NVFP4) {
+    p.gs_out = ep->gs_out;
+    p.out_scales = ep->out_scales;
+    p.out_kb_atoms = Nout / 64;
+  }
+  return NVFP4_OK;
+}
+
+// Split count of the split-K linear: as many splits as fit the output tiles once
+// on the SMs (at least one, at most one per K tile).
+int default_splits(int64_t M, int64_t N, int64_t K, int sms) {
+  const int64_t tiles = (M + gemm::BM - 1) / gemm::BM * ((N + gemm::BN - 1) / gemm::BN);
+  const int64_t k_tiles = K / gemm::BK;
+  int64_t s = tiles >= sms ? 1 : sms / tiles;
+  if (s > k_tiles) s = k_tiles;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
+// Launches the 1-CTA GEMM in split-K mode and the epilogue kernel on `p` (prepared
+// by prepare_linear); `splits` >= 1 and the workspace were checked by the caller.
+nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvfp4_operand_t *W, int splits,
+                             float *workspace, const DeviceInfo *dev, cudaStream_t st) {
+  using namespace gemm;
+  CUtensorMap tmA, tmB;
+  if (!make_codes_map(&tmA, A->codes, p.M, p.K) || !make_codes_map(&tmB, W->codes, p.N, p.K)) return NVFP4_ERR_CUDA;
+  p.kt_per_split = (p.k_tiles + splits - 1) / splits;
+  p.splits = (p.k_tiles + p.kt_per_split - 1) / p.kt_per_split;  // no empty split
+  p.partial = workspace;
+  p.tile_mode = MODE_NONE;
+  p.m_tiles = (p.M + BM - 1) / BM;
+  p.n_tiles = (p.N + BN - 1) / BN;
+  const int64_t units = int64_t(p.m_tiles) * p.n_tiles * p.splits;
+  if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
+  gemm_kernel<<<grid, NUM_THREADS, Plan1::BYTES, st>>>(tmA, tmB, p);
+  if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+  const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (p.M + 127) / 128 * 128 : p.M;
+  const int64_t threads = rows_cover * ((p.Nout + 63) / 64);
+  const int64_t blocks = (threads + REDUCE_THREADS - 1) / REDUCE_THREADS;
+  if (blocks > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  splitk_epilogue_kernel<<<static_cast<unsigned>(blocks), REDUCE_THREADS, 0, st>>>(p);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -241,101 +373,20 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
                             const nvfp4_segment_t *segs, int nseg, int epilogue, const nvfp4_epilogue_params_t *ep,
                             void *out, int out_kind, int64_t ldo, nvfp4_stream_t stream) {
   using namespace gemm;
-  if (!A || !W || !gs_a || !segs || !out) return NVFP4_ERR_INVALID_ARG;
-  if (!A->codes || !A->scales || !W->codes || !W->scales) return NVFP4_ERR_INVALID_ARG;
-  if (A->rows < 1 || W->rows < 1 || A->K < 1 || A->K != W->K) return NVFP4_ERR_INVALID_ARG;
-  if (epilogue < NVFP4_EPI_NONE || epilogue > NVFP4_EPI_GDN_GATES) return NVFP4_ERR_INVALID_ARG;
-  if (out_kind < NVFP4_OUT_BF16 || out_kind > NVFP4_OUT_NVFP4) return NVFP4_ERR_INVALID_ARG;
-  if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
-  const int64_t M = A->rows, N = W->rows, K = A->K;
-  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (K % BK != 0 || N % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  // segments: sorted, disjoint, 16-aligned, covering [0, N)
-  int64_t expect = 0;
-  for (int i = 0; i < nseg; ++i) {
-    if (!segs[i].gs_w || !aligned(segs[i].gs_w, 4)) return NVFP4_ERR_INVALID_ARG;
-    if (segs[i].n_begin != expect || segs[i].n_end <= segs[i].n_begin) return NVFP4_ERR_INVALID_ARG;
-    if (segs[i].n_begin % 16 != 0 || segs[i].n_end % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    expect = segs[i].n_end;
-  }
-  if (expect != N) return NVFP4_ERR_INVALID_ARG;
-  int64_t Nout = N;
-  if (epilogue == NVFP4_EPI_SILU_MUL) {
-    if (N % (2 * 128) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    Nout = N / 2;
-  }
-  if (epilogue == NVFP4_EPI_GDN_GATES) {
-    if (!ep || !ep->A_log || !ep->dt_bias || ep->n_heads < 1) return NVFP4_ERR_INVALID_ARG;
-    const int64_t h = ep->n_heads;
-    if (ep->beta_begin < 0 || ep->beta_begin + h > N || ep->alpha_begin < 0 || ep->alpha_begin + h > N)
-      return NVFP4_ERR_INVALID_ARG;
-    if (ep->beta_begin < ep->alpha_begin + h && ep->alpha_begin < ep->beta_begin + h) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned(ep->A_log, 4) || !aligned(ep->dt_bias, 4) || (ep->beta_out && !aligned(ep->beta_out, 4)) ||
-        (ep->g_out && !aligned(ep->g_out, 4)))
-      return NVFP4_ERR_MISALIGNED;
-  }
-  if (out_kind == NVFP4_OUT_NVFP4) {
-    if (!ep || !ep->gs_out || !ep->out_scales) return NVFP4_ERR_INVALID_ARG;
-    if (Nout % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned(out, 16) || !aligned(ep->out_scales, 16) || !aligned(ep->gs_out, 4)) return NVFP4_ERR_MISALIGNED;
-  } else {
-    const int64_t elem = out_kind == NVFP4_OUT_BF16 ? 2 : 4;
-    if (ldo < Nout) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned(out, 16) || (ldo * elem) % 16 != 0) return NVFP4_ERR_MISALIGNED;
-  }
-  if (!aligned(A->codes, 16) || !aligned(W->codes, 16) || !aligned(A->scales, 16) || !aligned(W->scales, 16) ||
-      !aligned(gs_a, 4))
-    return NVFP4_ERR_MISALIGNED;
-
+  Params p;
+  if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, p)) return st;
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;
+  const int64_t M = p.M, N = p.N, K = p.K;
 
   const bool pair = M > BM;  // 2-CTA tiles of 256 rows; one CTA per tile for M <= 128
   CUtensorMap tmA, tmB, tmSFA, tmSFB;
   if (!make_codes_map(&tmA, A->codes, M, K) || !make_codes_map(&tmB, W->codes, N, K)) return NVFP4_ERR_CUDA;
   if (pair && (!make_scales_map(&tmSFA, A->scales, M, K) || !make_scales_map(&tmSFB, W->scales, N, K)))
     return NVFP4_ERR_CUDA;
-
-  Params p{};
-  p.M = static_cast<int>(M);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
-  p.Nout = static_cast<int>(Nout);
-  p.mode = epilogue;
-  p.out_kind = out_kind;
   const int64_t tile_m = pair ? 2 * BM : BM;
   p.m_tiles = static_cast<int>((M + tile_m - 1) / tile_m);
-  p.n_tiles = epilogue == NVFP4_EPI_SILU_MUL ? static_cast<int>(Nout / 128) : static_cast<int>((N + BN - 1) / BN);
-  p.k_tiles = static_cast<int>(K / BK);
-  p.up_row0 = static_cast<int>(Nout);
-  p.kb_atoms = K / 64;
-  p.sfa = A->scales;
-  p.sfb = W->scales;
-  p.gs_a = gs_a;
-  p.nseg = nseg;
-  for (int i = 0; i < nseg; ++i) {
-    p.seg[i].n_begin = static_cast<int>(segs[i].n_begin);
-    p.seg[i].n_end = static_cast<int>(segs[i].n_end);
-    p.seg[i].gs_w = segs[i].gs_w;
-  }
-  p.out = out;
-  p.ldo = ldo;
-  p.beta_begin = p.alpha_begin = -1;
-  p.n_heads = 0;
-  if (epilogue == NVFP4_EPI_GDN_GATES) {
-    p.beta_begin = static_cast<int>(ep->beta_begin);
-    p.alpha_begin = static_cast<int>(ep->alpha_begin);
-    p.n_heads = static_cast<int>(ep->n_heads);
-    p.A_log = ep->A_log;
-    p.dt_bias = ep->dt_bias;
-    p.beta_out = ep->beta_out;
-    p.g_out = ep->g_out;
-  }
-  if (out_kind == NVFP4_OUT_NVFP4) {
-    p.gs_out = ep->gs_out;
-    p.out_scales = ep->out_scales;
-    p.out_kb_atoms = Nout / 64;
-  }
+  p.n_tiles = epilogue == NVFP4_EPI_SILU_MUL ? p.Nout / 128 : static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles;
   if (tiles > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -359,6 +410,35 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, gemm2_kernel, tmA, tmB, tmSFA, tmSFB, p) != cudaSuccess) return NVFP4_ERR_CUDA;
   return launch_status();
+}
+
+int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 16 || K < gemm::BK || K % gemm::BK != 0) return 0;
+  DeviceInfo *dev = nullptr;
+  if (current_device(&dev) != NVFP4_OK) return 0;
+  return default_splits(M, N, K, dev->sms);
+}
+
+size_t nvfp4_splitk_workspace_bytes(int64_t M, int64_t N, int split_k) {
+  if (M < 1 || N < 1 || split_k < 1 || M > kMaxDim || N > kMaxDim) return 0;
+  return static_cast<size_t>(M) * static_cast<size_t>(N) * static_cast<size_t>(split_k) * sizeof(float);
+}
+
+nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
+                                   const nvfp4_segment_t *segs, int nseg, int epilogue,
+                                   const nvfp4_epilogue_params_t *ep, void *out, int out_kind, int64_t ldo,
+                                   int split_k, void *workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  using namespace gemm;
+  Params p;
+  if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, p)) return st;
+  if (split_k < 1 || split_k > p.k_tiles) return NVFP4_ERR_INVALID_ARG;
+  if (!workspace) return NVFP4_ERR_INVALID_ARG;
+  if (workspace_bytes < nvfp4_splitk_workspace_bytes(p.M, p.N, split_k)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  return launch_splitk(p, A, W, split_k, static_cast<float *>(workspace), dev,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status_t nvfp4_get_device_status(int *code) {

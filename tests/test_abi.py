@@ -82,3 +82,12 @@ def test_invalid_arguments_rejected_without_launch(L):
     W_odd = nv.Operand(1 << 22, 1 << 23, 384, 512)
     segs384 = (nv.Segment * 1)(nv.Segment(0, 384, 1 << 24))
     assert call(A, W_odd, segs384, 1, 1, 0, 192) == 2                  # silu_mul needs N % 256
+
+
+def test_splitk_helpers_without_device(L):
+    assert L.nvfp4_splitk_workspace_bytes(32, 5120, 7) == 32 * 5120 * 7 * 4
+    assert L.nvfp4_splitk_workspace_bytes(0, 5120, 7) == 0
+    assert L.nvfp4_splitk_workspace_bytes(32, 5120, 0) == 0
+    # invalid sizes are rejected before any device query
+    assert L.nvfp4_splitk_default(0, 256, 512) == 0
+    assert L.nvfp4_splitk_default(8, 256, 300) == 0
