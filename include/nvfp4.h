@@ -218,6 +218,35 @@ NVFP4_API size_t nvfp4_splitk_workspace_bytes(int64_t M, int64_t N, int split_k)
 NVFP4_API int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K);
 
 /*
+ * nvfp4_linear_splitk_noalloc - nvfp4_linear_splitk for callers that cannot allocate
+ * device memory: the split-K partial sums go to a fixed scratch array inside the
+ * library instead of a caller workspace.  The pages have no counterpart of this entry
+ * point; it serves integrations whose interface hands the library only inputs and
+ * outputs (a plugin or custom-op hook with no workspace argument), or which must not
+ * allocate on the serving path, where cudaMalloc can synchronise the device and add
+ * latency.
+ *   Arguments and results as nvfp4_linear_splitk, without the workspace.  The call
+ *   allocates nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *   Scratch: NVFP4_NOALLOC_SCRATCH_BYTES of device memory held by every GPU that loads
+ *   the library until the process exits.  The first call on a device looks up the
+ *   array's device address (once per device, with that device current); make that
+ *   first call before any stream capture.  Every call shares the array and leaves
+ *   its contents behind; each call overwrites all of the scratch it reads, so no
+ *   state carries over, but calls that overlap on the GPU (other streams, other host
+ *   threads) race on it and must be serialised by the caller.
+ *   Errors: NVFP4_ERR_UNSUPPORTED_SHAPE when split_k * M * N * 4 bytes exceed
+ *   NVFP4_NOALLOC_SCRATCH_BYTES (use fewer splits or nvfp4_linear_splitk);
+ *   NVFP4_ERR_CUDA if the scratch address cannot be looked up; otherwise as
+ *   nvfp4_linear_splitk.
+ */
+#define NVFP4_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+NVFP4_API nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, const float *gs_a,
+                                                     const nvfp4_operand_t *W, const nvfp4_segment_t *segs,
+                                                     int nseg, int epilogue, const nvfp4_epilogue_params_t *ep,
+                                                     void *out, int out_kind, int64_t ldo, int split_k,
+                                                     nvfp4_stream_t stream);
+
+/*
  * nvfp4_get_device_status - read and clear the device status word of the current
  * device.  Kernels never spin forever: every wait on an mbarrier has an iteration
  * limit, and a wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the

@@ -14,7 +14,8 @@ from typing import Optional, Sequence
 
 __all__ = [
     "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
-    "linear_splitk", "splitk_default", "splitk_workspace_bytes",
+    "linear_splitk", "linear_splitk_noalloc", "splitk_default", "splitk_workspace_bytes",
+    "NOALLOC_SCRATCH_BYTES",
     "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
 ]
 
@@ -24,6 +25,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4_w4a4.so")
 EPILOGUES = {"none": 0, "silu_mul": 1, "gdn_gates": 2}
 OUT_KINDS = {"bf16": 0, "f32": 1, "nvfp4": 2}
 MAX_SEGMENTS = 16
+NOALLOC_SCRATCH_BYTES = 8 << 20  # NVFP4_NOALLOC_SCRATCH_BYTES of include/nvfp4.h
 
 _c_i64 = ctypes.c_int64
 _c_vp = ctypes.c_void_p
@@ -52,7 +54,7 @@ class NVFP4Error(RuntimeError):
 _LIB = None
 SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
            "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
-           "nvfp4_splitk_default", "nvfp4_get_device_status")
+           "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_get_device_status")
 
 
 def lib():
@@ -88,6 +90,11 @@ def lib():
     L.nvfp4_splitk_workspace_bytes.argtypes = [_c_i64, _c_i64, ctypes.c_int]
     L.nvfp4_splitk_default.restype = ctypes.c_int
     L.nvfp4_splitk_default.argtypes = [_c_i64, _c_i64, _c_i64]
+    L.nvfp4_linear_splitk_noalloc.restype = ctypes.c_int
+    L.nvfp4_linear_splitk_noalloc.argtypes = [ctypes.POINTER(Operand), _c_vp, ctypes.POINTER(Operand),
+                                              ctypes.POINTER(Segment), ctypes.c_int, ctypes.c_int,
+                                              ctypes.POINTER(EpilogueParams), _c_vp, ctypes.c_int, _c_i64,
+                                              ctypes.c_int, _c_vp]
     L.nvfp4_get_device_status.restype = ctypes.c_int
     L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     _LIB = L
@@ -269,6 +276,25 @@ def linear_splitk(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] =
     _check(lib().nvfp4_linear_splitk(*args, int(split_k), _c_vp(workspace.data_ptr()),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
            "nvfp4_linear_splitk")
+    return result
+
+
+def linear_splitk_noalloc(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None,
+                          epilogue: str = "none", out_dtype: str = "bf16", out=None, ldo: Optional[int] = None,
+                          gates: Optional[dict] = None, gs_out=None, out_scales=None,
+                          split_k: Optional[int] = None, stream=None):
+    """``linear_splitk`` whose partial sums live in the library's fixed scratch array
+    (``NOALLOC_SCRATCH_BYTES``), for callers that cannot hand in a workspace.
+
+    The library allocates nothing for it (the output buffers allocated here when
+    ``out`` / ``out_scales`` are None are this wrapper's, not the entry point's).
+    Calls that overlap on the GPU share the scratch and race: serialise them.
+    """
+    M, N, K = a.rows, w.rows, a.cols
+    if split_k is None:
+        split_k = splitk_default(M, N, K)
+    args, result, _keep = _linear_args(a, w, segments, epilogue, out_dtype, out, ldo, gates, gs_out, out_scales)
+    _check(lib().nvfp4_linear_splitk_noalloc(*args, int(split_k), _stream(stream)), "nvfp4_linear_splitk_noalloc")
     return result
 
 

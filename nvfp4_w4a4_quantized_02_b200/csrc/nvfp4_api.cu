@@ -285,6 +285,31 @@ nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvf
   return launch_status();
 }
 
+// ------------------------------------------------- scratch for callers that cannot allocate
+// nvfp4_linear_splitk_noalloc keeps its split-K partial sums in this fixed array, so
+// that callers which cannot allocate device memory (no workspace to hand in) can
+// still run the decode-regime linear.  Every GPU that loads the library holds these
+// NVFP4_NOALLOC_SCRATCH_BYTES until the process exits.
+static __device__ __align__(256) float g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+// Device address of g_noalloc_scratch on each device, looked up once per device (the
+// host-side name of the array is not a device address).
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+nvfp4_status_t noalloc_scratch(float **ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NVFP4_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<float *>(p);
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return NVFP4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -439,6 +464,23 @@ nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const float *gs_a, 
   if (nvfp4_status_t st = current_device(&dev)) return st;
   return launch_splitk(p, A, W, split_k, static_cast<float *>(workspace), dev,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
+                                           const nvfp4_segment_t *segs, int nseg, int epilogue,
+                                           const nvfp4_epilogue_params_t *ep, void *out, int out_kind, int64_t ldo,
+                                           int split_k, nvfp4_stream_t stream) {
+  using namespace gemm;
+  Params p;
+  if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, p)) return st;
+  if (split_k < 1 || split_k > p.k_tiles) return NVFP4_ERR_INVALID_ARG;
+  if (nvfp4_splitk_workspace_bytes(p.M, p.N, split_k) > NVFP4_NOALLOC_SCRATCH_BYTES)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;  // the partials do not fit the fixed scratch array
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  float *scratch = nullptr;
+  if (nvfp4_status_t st = noalloc_scratch(&scratch)) return st;
+  return launch_splitk(p, A, W, split_k, scratch, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status_t nvfp4_get_device_status(int *code) {
