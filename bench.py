@@ -15,6 +15,8 @@ One JSON line on stdout (rank 0).  Workloads (``--workload``):
 * ``sweep``: all 496 linears of the 64-layer hybrid model (48 GDN layers x 2 GEMMs,
   16 attention layers x 2 GEMMs with q|k|v fused, 64 MLPs x 2 GEMMs with gate|up
   fused), each fed by the NVFP4 quantiser, at ``--M`` prefill tokens.
+* ``decode``: the same 496 linears for one decode step of ``--M`` (default 32)
+  sequences through the split-K linear (weight-bandwidth bound).
 
 Multi-GPU (torchrun): every rank runs the same workload on its own GPU with its own
 inputs (independent token batches, weak scaling); no collective touches the data
@@ -305,6 +307,17 @@ class Workload:
         raise NotImplementedError
 
     cpu_sample_note = ""
+    use_graph = False  # replay the step as a CUDA graph (launch-bound workloads)
+
+    def plan(self, x):
+        """The step as a list of (phase, launch) pairs; every launch writes preallocated buffers."""
+        raise NotImplementedError
+
+    def step(self, tm=NO_TIMER, x=None):
+        for phase, launch in self.plan(self.x if x is None else x):
+            with tm(phase):
+                launch()
+        return self.out
 
 
 class MLPBlock(Workload):
@@ -353,19 +366,18 @@ class MLPBlock(Workload):
         return {"M": self.M, "hidden": self.H, "intermediate": self.I,
                 "step": "global_scale+quantize(X) -> gate|up GEMM (SiLU*mul, NVFP4 requant) -> down GEMM (BF16)"}
 
-    def step(self, tm=NO_TIMER, x=None):
+    def plan(self, x):
         nv = self.nv
-        x = self.x if x is None else x
-        with tm("global_scale"):
-            nv.global_scale(x, out=self.gs_x)
-        with tm("quantize"):
-            xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
-        with tm("gemm_gate_up"):
-            hq = nv.linear(xq, self.w_gu, segments=self.seg_gu, epilogue="silu_mul", out_dtype="nvfp4",
-                           gs_out=self.gs_h, out=self.h_codes, out_scales=self.h_scales)
-        with tm("gemm_down"):
-            nv.linear(hq, self.w_d, out_dtype="bf16", out=self.out)
-        return self.out
+        xq = nv.NVFP4Tensor(self.xq_codes, self.xq_scales, self.gs_x, self.M, self.H)
+        hq = nv.NVFP4Tensor(self.h_codes, self.h_scales, self.gs_h, self.M, self.I)
+        return [
+            ("global_scale", lambda: nv.global_scale(x, out=self.gs_x)),
+            ("quantize", lambda: nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)),
+            ("gemm_gate_up", lambda: nv.linear(xq, self.w_gu, segments=self.seg_gu, epilogue="silu_mul",
+                                               out_dtype="nvfp4", gs_out=self.gs_h, out=self.h_codes,
+                                               out_scales=self.h_scales)),
+            ("gemm_down", lambda: nv.linear(hq, self.w_d, out_dtype="bf16", out=self.out)),
+        ]
 
     cpu_sample_note = ("MLP-block sample (32 token rows, 256 intermediate channels, K=5120; global scale + "
                        "quantise + gate|up + SiLU*mul + requant + down); numpy FP64 oracle")
@@ -402,11 +414,8 @@ class QuantizeOnly(Workload):
         return {"M": self.M, "K": self.K, "gs": "static (calibrated once from amax)",
                 "bytes_per_element": 2.5625}
 
-    def step(self, tm=NO_TIMER, x=None):
-        x = self.x if x is None else x
-        with tm("quantize"):
-            self.nv.quantize(x, self.gs, codes=self.codes, scales=self.scales)
-        return self.codes
+    def plan(self, x):
+        return [("quantize", lambda: self.nv.quantize(x, self.gs, codes=self.codes, scales=self.scales))]
 
     def extra(self, torch):
         """Dynamic mode (amax pass + finalize + quantise), timed separately after the main region."""
@@ -472,17 +481,15 @@ class GDNInProj(Workload):
                 "step": "global_scale+quantize(X) -> fused GEMM (per-segment alpha, sigmoid beta, "
                         "-exp(A_log)*softplus(a+dt_bias)) -> BF16 + FP32 gates"}
 
-    def step(self, tm=NO_TIMER, x=None):
+    def plan(self, x):
         nv = self.nv
-        x = self.x if x is None else x
-        with tm("global_scale"):
-            nv.global_scale(x, out=self.gs_x)
-        with tm("quantize"):
-            xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
-        with tm("gemm"):
-            nv.linear(xq, self.w, segments=self.segs, epilogue="gdn_gates", gates=self.gates,
-                      out_dtype="bf16", out=self.out)
-        return self.out
+        xq = nv.NVFP4Tensor(self.xq_codes, self.xq_scales, self.gs_x, self.M, self.K)
+        return [
+            ("global_scale", lambda: nv.global_scale(x, out=self.gs_x)),
+            ("quantize", lambda: nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)),
+            ("gemm", lambda: nv.linear(xq, self.w, segments=self.segs, epilogue="gdn_gates", gates=self.gates,
+                                       out_dtype="bf16", out=self.out)),
+        ]
 
     cpu_sample_note = ("GDN in-proj sample: 32 token rows x 320 weight rows (64 each of q/k/v/z + 32 beta + "
                        "32 alpha), K=5120; quantise X + fused linear + gates; numpy FP64 oracle")
@@ -520,16 +527,14 @@ class SmallLinear(Workload):
         return {"M": self.M, "N": self.N, "K": self.K,
                 "step": "global_scale+quantize(X) -> GEMM -> BF16"}
 
-    def step(self, tm=NO_TIMER, x=None):
+    def plan(self, x):
         nv = self.nv
-        x = self.x if x is None else x
-        with tm("global_scale"):
-            nv.global_scale(x, out=self.gs_x)
-        with tm("quantize"):
-            xq = nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)
-        with tm("gemm"):
-            nv.linear(xq, self.w, out_dtype="bf16", out=self.out)
-        return self.out
+        xq = nv.NVFP4Tensor(self.xq_codes, self.xq_scales, self.gs_x, self.M, self.K)
+        return [
+            ("global_scale", lambda: nv.global_scale(x, out=self.gs_x)),
+            ("quantize", lambda: nv.quantize(x, self.gs_x, codes=self.xq_codes, scales=self.xq_scales)),
+            ("gemm", lambda: nv.linear(xq, self.w, out_dtype="bf16", out=self.out)),
+        ]
 
     cpu_sample_note = "the whole linear (128 x 1024 x 1024): quantise X + dequantise-then-FP64 matmul"
 
@@ -638,39 +643,43 @@ class HybridSweep(Workload):
                 "gemm_launches_per_step": 256, "packed_weight_gib": round(self.packed_bytes / 2**30, 3),
                 "step": "per layer: quantise(input) -> fused NVFP4 GEMM(s) with the layer's epilogue"}
 
-    def step(self, tm=NO_TIMER, x=None):
+    def plan(self, x):
         nv = self.nv
-        x = self.x if x is None else x
-        qx = None
-        for li, L in enumerate(self.layers):
-            with tm("quantize"):
-                qx = nv.quantize(x, self.gs_x, codes=self.qx[0], scales=self.qx[1])
+        H, I, M = 5120, 17408, self.M
+        qx = nv.NVFP4Tensor(self.qx[0], self.qx[1], self.gs_x, M, H)
+        qgc = nv.NVFP4Tensor(self.qgc[0], self.qgc[1], self.gs_gc, M, 4096)
+        qac = nv.NVFP4Tensor(self.qac[0], self.qac[1], self.gs_ac, M, 6144)
+        hq = nv.NVFP4Tensor(self.hq[0], self.hq[1], self.gs_h, M, I)
+        quant_x = ("quantize", lambda: nv.quantize(x, self.gs_x, codes=self.qx[0], scales=self.qx[1]))
+        out = []
+        for L in self.layers:
+            out.append(quant_x)
             if "qkv" in L:
                 w, segs = L["qkv"]
-                with tm("gemm_attn_qkv"):
-                    nv.linear(qx, w, segments=segs, out_dtype="bf16", out=self.out_qkv)
-                with tm("quantize"):
-                    qc = nv.quantize(self.x_attn_core, self.gs_ac, codes=self.qac[0], scales=self.qac[1])
-                with tm("gemm_attn_o"):
-                    nv.linear(qc, L["o"], out_dtype="bf16", out=self.out)
+                out.append(("gemm_attn_qkv", lambda w=w, segs=segs: self._lin(
+                    qx, w, segments=segs, out_dtype="bf16", out=self.out_qkv)))
+                out.append(("quantize", lambda: nv.quantize(self.x_attn_core, self.gs_ac, codes=self.qac[0],
+                                                            scales=self.qac[1])))
+                out.append(("gemm_attn_o", lambda wo=L["o"]: self._lin(qac, wo, out_dtype="bf16", out=self.out)))
             else:
                 w, segs = L["in"]
-                with tm("gemm_gdn_in"):
-                    nv.linear(qx, w, segments=segs, epilogue="gdn_gates", gates=self.gates, out_dtype="bf16",
-                              out=self.out_gdn)
-                with tm("quantize"):
-                    qc = nv.quantize(self.x_gdn_core, self.gs_gc, codes=self.qgc[0], scales=self.qgc[1])
-                with tm("gemm_gdn_out"):
-                    nv.linear(qc, L["out"], out_dtype="bf16", out=self.out)
-            with tm("quantize"):
-                qx = nv.quantize(x, self.gs_x, codes=self.qx[0], scales=self.qx[1])
+                out.append(("gemm_gdn_in", lambda w=w, segs=segs: self._lin(
+                    qx, w, segments=segs, epilogue="gdn_gates", gates=self.gates, out_dtype="bf16",
+                    out=self.out_gdn)))
+                out.append(("quantize", lambda: nv.quantize(self.x_gdn_core, self.gs_gc, codes=self.qgc[0],
+                                                            scales=self.qgc[1])))
+                out.append(("gemm_gdn_out", lambda wo=L["out"]: self._lin(qgc, wo, out_dtype="bf16",
+                                                                          out=self.out)))
+            out.append(quant_x)
             w, segs = L["gu"]
-            with tm("gemm_gate_up"):
-                hq = nv.linear(qx, w, segments=segs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=self.gs_h,
-                               out=self.hq[0], out_scales=self.hq[1])
-            with tm("gemm_down"):
-                nv.linear(hq, L["down"], out_dtype="bf16", out=self.out)
-        return self.out
+            out.append(("gemm_gate_up", lambda w=w, segs=segs: self._lin(
+                qx, w, segments=segs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=self.gs_h, out=self.hq[0],
+                out_scales=self.hq[1])))
+            out.append(("gemm_down", lambda wd=L["down"]: self._lin(hq, wd, out_dtype="bf16", out=self.out)))
+        return out
+
+    def _lin(self, a, w, **kw):
+        return self.nv.linear(a, w, **kw)
 
     cpu_sample_note = ("one sampled MLP block and one sampled GDN in-proj (32 token rows, 256-320 weight rows, "
                        "full K), FLOP-weighted; numpy FP64 oracle")
@@ -681,8 +690,58 @@ class HybridSweep(Workload):
         return f1 + f2, s1 + s2
 
 
+class DecodeSweep(HybridSweep):
+    """One decode step of the 496 linears for a batch of M sequences (concurrency 32 by
+    default): the split-K linear streams every weight once per step from HBM, so the
+    bound is HBM bandwidth over the packed weights.  The step's 704 launches are
+    replayed as one CUDA graph (launch overhead would otherwise dominate)."""
+    use_graph = True
+
+    def __init__(self, nv, M=32, seed=0):
+        import torch
+        super().__init__(nv, M=M, seed=seed)
+        self.name = f"decode_sweep_496_linears_m{M}"
+        shapes = [(12352, 5120), (5120, 4096), (8192, 5120), (5120, 6144), (34816, 5120), (5120, 17408)]
+        ws = max(nv.splitk_workspace_bytes(M, n, nv.splitk_default(M, n, k)) for n, k in shapes)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device="cuda")
+        self.splits = {f"{n}x{k}": nv.splitk_default(M, n, k) for n, k in shapes}
+        self.launches_per_step = 48 * 4 + 16 * 4 + 64 * 3 + 256  # + one split-K epilogue launch per GEMM
+        H, I = 5120, 17408
+        wb = lambda n, k: n * k * 0.5625  # packed codes + scales
+
+        def gemm_bytes(n, k, count):
+            return count * (wb(n, k) + M * k * 0.5625 + M * n * 2)
+        self.bytes_gu = wb(2 * I, H) + M * H * 0.5625 + M * I * 0.5625
+        self.dominant = ("gemm_gate_up", self.bytes_gu, "hbm",
+                         f"nvfp4_linear_splitk (MLP gate|up, SiLU*mul, NVFP4 requant; "
+                         f"split_k {self.splits['34816x5120']})")
+        self.phases = {"quantize": ("GB/s", 2.5625 * M * (128 * H + 48 * 4096 + 16 * 6144)),
+                       "gemm_gdn_in": ("GB/s", gemm_bytes(12352, H, 48)),
+                       "gemm_gdn_out": ("GB/s", gemm_bytes(H, 4096, 48)),
+                       "gemm_attn_qkv": ("GB/s", gemm_bytes(8192, H, 16)),
+                       "gemm_attn_o": ("GB/s", gemm_bytes(H, 6144, 16)),
+                       "gemm_gate_up": ("GB/s", 64 * self.bytes_gu),
+                       "gemm_down": ("GB/s", gemm_bytes(H, I, 64))}
+        self.l2_note = (f"weights {self.packed_bytes / 2**30:.2f} GiB packed, streamed from HBM once per step "
+                        "(> L2)")
+
+    def config(self):
+        c = super().config()
+        c["split_k"] = self.splits
+        c["step"] = ("per layer: quantise(input) -> split-K NVFP4 GEMM(s) -> split-K epilogue kernel "
+                     "(the layer's epilogue)")
+        return c
+
+    def _lin(self, a, w, **kw):
+        return self.nv.linear_splitk(a, w, workspace=self.workspace, **kw)
+
+    def report(self, ms_step):
+        return {"decode_step": {"ms": round(ms_step, 4), "tokens_per_s_linears_only": round(self.M / ms_step * 1e3, 1),
+                                "weight_GB/s": round(self.packed_bytes / ms_step / 1e6, 1)}}
+
+
 WORKLOADS = {"mlp": MLPBlock, "quantize": QuantizeOnly, "gdn": GDNInProj, "linear": SmallLinear,
-             "sweep": HybridSweep}
+             "sweep": HybridSweep, "decode": DecodeSweep}
 
 
 def make_workload(args, nv):
@@ -694,6 +753,28 @@ def make_workload(args, nv):
 
 
 # ---------------------------------------------------------------- GPU arm
+def capture_graph(torch, launches):
+    """One CUDA graph holding ``launches`` (callables that launch on the current stream)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for launch in launches:
+            launch()
+    return g
+
+
+def time_replays(torch, g, n):
+    """Device time of ``n`` back-to-back replays of graph ``g`` (CUDA events), in ms."""
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(n):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
 def run_ours(args, ws, rank):
     import torch
     import nvfp4_w4a4_quantized_02_b200 as nv
@@ -705,6 +786,7 @@ def run_ours(args, ws, rank):
     nv.lib()
     peaks, peak_src = load_peaks()
     wl = make_workload(args, nv)
+    graph = wl.use_graph or args.graph
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda") if wl.flush_l2 else None
 
@@ -713,8 +795,14 @@ def run_ours(args, ws, rank):
         if flush is not None:
             flush.zero_()
     torch.cuda.synchronize()
+    plan = wl.plan(wl.x)
+    g_step = capture_graph(torch, [launch for _, launch in plan]) if graph else None
+    if graph:
+        for _ in range(2):
+            g_step.replay()
+        torch.cuda.synchronize()
 
-    tm = KernelTimer(torch)
+    tm = KernelTimer(torch) if not graph else NO_TIMER
     steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
@@ -729,7 +817,10 @@ def run_ours(args, ws, rank):
     start.record(stream)
     for i in range(args.steps):
         steps[i][0].record(stream)
-        wl.step(tm)
+        if graph:
+            g_step.replay()
+        else:
+            wl.step(tm)
         steps[i][1].record(stream)
         if flush is not None:
             flush.zero_()
@@ -744,13 +835,26 @@ def run_ours(args, ws, rank):
         elapsed_ms = max_over_ranks(elapsed_ms, "cuda")
         torch.distributed.barrier()
 
-    ksum = tm.summary()
+    # per-phase device time: events around each launch (eager), or one graph per phase
+    # holding that phase's launches of one step (graph mode: no host gaps between them)
+    per_phase = {}
+    if graph:
+        for key in wl.phases:
+            launches = [launch for ph, launch in plan if ph == key]
+            if launches:
+                g = capture_graph(torch, launches)
+                reps = 5
+                per_phase[key] = {"launches": len(launches), "ms_step": time_replays(torch, g, reps) / reps}
+                del g
+    else:
+        for key, d in tm.summary().items():
+            per_phase[key] = {"launches": d["launches"] // args.steps, "ms_step": d["ms_total"] / args.steps}
     kernels = {}
     for key, (unit, amount) in wl.phases.items():
-        if key not in ksum:
+        if key not in per_phase:
             continue
-        ms = ksum[key]["ms_total"] / args.steps
-        d = {"launches_per_step": ksum[key]["launches"] // args.steps, "ms_per_step": round(ms, 5)}
+        ms = per_phase[key]["ms_step"]
+        d = {"launches_per_step": per_phase[key]["launches"], "ms_per_step": round(ms, 5)}
         if unit == "GB/s":
             d["GB/s"] = round(amount / ms / 1e6, 1)
             d["frac_hbm"] = round(d["GB/s"] / peaks["hbm_gbs"], 4)
@@ -760,7 +864,7 @@ def run_ours(args, ws, rank):
         kernels[key] = d
 
     key, per_launch, bound, label = wl.dominant
-    avg_ms = ksum[key]["ms_avg"]
+    avg_ms = per_phase[key]["ms_step"] / per_phase[key]["launches"]
     if bound == "hbm":
         achieved = per_launch / avg_ms / 1e6
         peak, unit = peaks["hbm_gbs"], "GB/s"
@@ -771,16 +875,18 @@ def run_ours(args, ws, rank):
         note = f"{peak_src} bf16_tflops_sustained x {FP4_OVER_BF16} (nominal FP4/BF16 ratio)"
     roof = {"kernel": label, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": load_traffic(f"{key}@{wl.name}"),
-            "avg_launch_ms": round(avg_ms, 5), "work_per_launch": per_launch, "peak_note": note}
+            "avg_launch_ms": round(avg_ms, 5), "work_per_launch": per_launch, "peak_note": note,
+            "timing": "graph of the phase's launches, CUDA events" if graph else "CUDA events per launch"}
 
-    e2e = run_e2e(wl, args, torch, flush)
+    e2e = run_e2e(wl, args, torch, flush, g_step)
     ms = elapsed_ms / args.steps
     if wl.unit == "GB/s":
         value = ws * wl.work() / (ms * 1e-3) / 1e9
     else:
         value = ws * wl.work() / (ms * 1e-3) / 1e12
     cfg = {"workload": wl.name, **wl.config(),
-           "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU", "l2": wl.l2_note}
+           "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU", "l2": wl.l2_note,
+           "launch": "one CUDA graph per step" if graph else "eager launches"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -790,29 +896,39 @@ def run_ours(args, ws, rank):
     }
     if hasattr(wl, "extra"):
         line["kernels"].update(wl.extra(torch))
+    if hasattr(wl, "report"):
+        line["kernels"].update(wl.report(ms))
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(wl, args, torch, flush):
+def run_e2e(wl, args, torch, flush, g_step=None):
     """The same step through the public API with host buffers: pinned H2D of the step's
-    input, the step, D2H of its result, all inside the timed region."""
+    input, the step, D2H of its result, all inside the timed region.  A graph step reads
+    the buffer it was captured with, so the input is copied into that buffer."""
     stream = torch.cuda.current_stream()
     x_host = wl.x.cpu().pin_memory()
     out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
-    x_dev = torch.empty_like(wl.x)
+    x_dev = wl.x if g_step is not None else torch.empty_like(wl.x)
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        if g_step is not None:
+            g_step.replay()
+            out_host.copy_(wl.out, non_blocking=True)
+        else:
+            out_host.copy_(wl.step(x=x_dev), non_blocking=True)
+
     n = max(1, min(args.steps, 10))
     for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        out_host.copy_(wl.step(x=x_dev), non_blocking=True)
+        one()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     for a, b in evs:
         a.record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        out_host.copy_(wl.step(x=x_dev), non_blocking=True)
+        one()
         b.record(stream)
         if flush is not None:
             flush.zero_()
@@ -906,14 +1022,16 @@ class _CpuOnly:
         self.unit = cls.unit
         self.cpu_sample_note = cls.cpu_sample_note
         obj = object.__new__(cls)
-        obj.M = args.M or {"mlp": 32768, "quantize": 32768, "gdn": 8192, "linear": 128, "sweep": 32768}[args.workload]
+        obj.M = args.M or {"mlp": 32768, "quantize": 32768, "gdn": 8192, "linear": 128, "sweep": 32768,
+                           "decode": 32}[args.workload]
         obj.K = {"quantize": 5120, "gdn": 5120, "linear": 1024}.get(args.workload, 5120)
         obj.N = {"linear": 1024, "gdn": 12352}.get(args.workload, 0)
         obj.flops = 2.0 * obj.M * obj.N * obj.K
         self.obj = obj
         self.name = {"mlp": f"mlp_block_m{obj.M}_h5120_i17408", "quantize": f"quantize_m{obj.M}_k5120",
                      "gdn": f"gdn_inproj_m{obj.M}_n12352_k5120", "linear": f"linear_m{obj.M}_n1024_k1024",
-                     "sweep": f"hybrid_sweep_496_linears_m{obj.M}"}[args.workload]
+                     "sweep": f"hybrid_sweep_496_linears_m{obj.M}",
+                     "decode": f"decode_sweep_496_linears_m{obj.M}"}[args.workload]
 
     def cpu_sample(self):
         return self.cls.cpu_sample(self.obj)
@@ -954,6 +1072,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mlp")
     ap.add_argument("--M", type=int, default=0, help="token rows (default: the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="replay each step as one CUDA graph")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":

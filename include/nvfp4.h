@@ -195,7 +195,8 @@ NVFP4_API nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_
  *   Source: the blog's results section (結果: decode at concurrency 32, 1,154 tok/s
  *   against 621 tok/s in BF16) is the regime; the method is nvfp4_linear's.
  *   Arguments as nvfp4_linear, plus:
- *   split_k: 1 .. K/256 (nvfp4_splitk_default gives the library's choice);
+ *   split_k: 1 .. K/256 (nvfp4_splitk_default gives the library's choice); with 1
+ *   the call runs nvfp4_linear itself and does not touch the workspace;
  *   workspace: device, >= nvfp4_splitk_workspace_bytes(M, N, split_k) bytes,
  *   16-byte aligned, owned by the caller; its contents on entry do not matter and
  *   are overwritten.  Two calls that share a workspace must not overlap on the GPU.
@@ -213,8 +214,10 @@ NVFP4_API nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const flo
 NVFP4_API size_t nvfp4_splitk_workspace_bytes(int64_t M, int64_t N, int split_k);
 
 /* The split count the library would choose for an M x N x K linear on the current
- * device: enough units to fill the SMs once (>= 1, <= K/256).  0 for invalid sizes
- * or when the device cannot be queried. */
+ * device (>= 1, <= K/256): 1 unless the output tiles fill under a quarter of the SMs
+ * and K has at least 32 tiles of 256; then enough units to fill the SMs once, with at
+ * least 8 K tiles per split.  0 for invalid sizes or when the device cannot be
+ * queried. */
 NVFP4_API int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K);
 
 /*

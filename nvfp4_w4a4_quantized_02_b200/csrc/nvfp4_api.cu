@@ -249,13 +249,18 @@ nvfp4_status_t prepare_linear(const nvfp4_operand_t *A, const float *gs_a, const
   return NVFP4_OK;
 }
 
-// Split count of the split-K linear: as many splits as fit the output tiles once
-// on the SMs (at least one, at most one per K tile).
+// Split count of the split-K linear.  Splitting pays only when few output tiles would
+// leave most SMs idle for a long K loop: the partial sums and the second kernel cost
+// about as much as a short GEMM (measured at 32 rows: the 5120 x 17408 projection gains
+// with 7 splits; 12352 x 5120, 5120 x 4096 and 5120 x 6144 lose).  So: more than one
+// split only when the tiles fill under a quarter of the SMs and K has >= 32 tiles; then
+// as many splits as fill the SMs once, keeping >= 8 K tiles per split.
 int default_splits(int64_t M, int64_t N, int64_t K, int sms) {
   const int64_t tiles = (M + gemm::BM - 1) / gemm::BM * ((N + gemm::BN - 1) / gemm::BN);
   const int64_t k_tiles = K / gemm::BK;
-  int64_t s = tiles >= sms ? 1 : sms / tiles;
-  if (s > k_tiles) s = k_tiles;
+  if (tiles * 4 >= sms || k_tiles < 32) return 1;
+  int64_t s = sms / tiles;
+  if (s > k_tiles / 8) s = k_tiles / 8;
   return static_cast<int>(s < 1 ? 1 : s);
 }
 
@@ -460,6 +465,8 @@ nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const float *gs_a, 
   if (!workspace) return NVFP4_ERR_INVALID_ARG;
   if (workspace_bytes < nvfp4_splitk_workspace_bytes(p.M, p.N, split_k)) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return NVFP4_ERR_MISALIGNED;
+  if (split_k == 1)  // one split: the ordinary kernel, without partials or the second kernel
+    return nvfp4_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, stream);
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;
   return launch_splitk(p, A, W, split_k, static_cast<float *>(workspace), dev,

@@ -37,7 +37,9 @@ def test_down_proj_decode_full_size(nv):
     a = nv.quantize(to_dev_bf16(xb))
     w = nv.quantize(to_dev_bf16(wb))
     s_def = nv.splitk_default(M, N, K)
-    assert 1 <= s_def <= K // 256
+    assert 1 < s_def <= K // 256  # 20 output tiles, 68 K tiles: the split pays here
+    assert nv.splitk_default(M, 34816, 5120) == 1  # 136 tiles already fill the SMs
+    assert nv.splitk_default(M, 5120, 4096) == 1  # 16 K tiles: too short to split
     for s in (s_def, 1, 5):
         y32 = nv.linear_splitk(a, w, out_dtype="f32", split_k=s)
         y16 = nv.linear_splitk(a, w, out_dtype="bf16", split_k=s)
