@@ -32,6 +32,11 @@ R3  the linear: Y[m, n] = alpha(n) * sum_k Ahat[m, k] * What[n, k] with
 R4  epilogues in FP64: SiLU(gate) * up; beta = sigmoid; g = -exp(A_log) * softplus(a + dt_bias)
     with softplus(x) = max(x, 0) + log1p(exp(-|x|)).
 R5  re-quantising an output for the next layer first rounds it to BF16 (nearest even).
+R12 fused-group repair (blog section 罠①: the fused group is rewritten to a common
+    global scale and the ratio is folded into the block scales, re-rounding error
+    <= 6.2 %): the common scale is the smallest segment scale, gs_c = min gs_seg, so
+    every ratio is <= 1 and no block scale saturates; each block scale becomes
+    sf' = E4M3(fl32(dec(sf) * fl32(gs_c / gs_seg))), nearest even; codes are kept.
 
 Float32 steps (R1, R2) use numpy float32 scalars/arrays, whose +, *, / are IEEE-754
 single precision, round to nearest even: the same operations a correct kernel
@@ -47,6 +52,7 @@ __all__ = [
     "e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode",
     "global_scale", "quantize", "dequantize", "block_scaled_matmul", "linear",
     "silu", "sigmoid", "softplus", "silu_mul", "gdn_gates", "round_to_bf16",
+    "fold_segments",
 ]
 
 E2M1_MAX = 6.0
@@ -247,3 +253,22 @@ def round_to_bf16(x) -> np.ndarray:
     x = np.asarray(x, dtype=np.float64)
     m, e = np.frexp(x)                    # x = m * 2**e, 0.5 <= |m| < 1
     return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+# ------------------------------------------------------------ fused-group repair
+def fold_segments(sf_segments, gs_segments):
+    """Re-express the modules of a fused weight with one global scale (reading R12).
+
+    ``sf_segments``: list of logical block-scale arrays (uint8 [rows_i, cols/16]), one per
+    module; ``gs_segments``: the modules' global scales.  Returns ``(sf_folded_list, gs_c)``.
+    The value a block decodes to, e2m1 * dec(sf') / gs_c, then differs from
+    e2m1 * dec(sf) / gs_seg only by the re-rounding of the E4M3 scale.
+    """
+    gs = [np.float32(g) for g in gs_segments]
+    gs_c = np.float32(min(gs))
+    out = []
+    for sf, g in zip(sf_segments, gs):
+        ratio = np.float32(gs_c / g)                      # one fl32 division
+        s = (e4m3_decode(sf).astype(np.float32) * ratio).astype(np.float32)
+        out.append(e4m3_encode(s))
+    return out, gs_c

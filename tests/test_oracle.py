@@ -351,3 +351,79 @@ def test_synth_is_seeded_and_bf16():
     t = synth.student_t_activations(16, 128, seed=0)
     x = synth.bf16_to_f32(t)
     assert np.all(np.isfinite(x))
+
+
+# ------------------------------------------------------------ fused-group repair
+def _rand_sf(rng, shape, lo=0x08, hi=0x7E):
+    return rng.integers(lo, hi + 1, shape).astype(np.uint8)
+
+
+def test_fold_equal_scales_is_identity():
+    rng = np.random.default_rng(100)
+    sfs = [_rand_sf(rng, (8, 4)), _rand_sf(rng, (16, 4))]
+    out, gs_c = oracle.fold_segments(sfs, [3.5, 3.5])
+    assert gs_c == np.float32(3.5)
+    for a, b in zip(sfs, out):
+        assert np.array_equal(a, b)
+
+
+def test_fold_power_of_two_ratio_is_exact():
+    """gs_seg = 4 * gs_c: every normal scale that stays normal is divided by 4 exactly."""
+    rng = np.random.default_rng(101)
+    sf = _rand_sf(rng, (32, 8), lo=0x20, hi=0x7E)   # >= 2**-3: /4 stays >= 2**-5, normal
+    out, gs_c = oracle.fold_segments([sf, sf], [2.0, 8.0])
+    assert gs_c == np.float32(2.0)
+    assert np.array_equal(out[0], sf)
+    assert np.array_equal(oracle.e4m3_decode(out[1]), oracle.e4m3_decode(sf) / 4.0)
+
+
+def test_fold_rerounding_bound_matches_the_pages():
+    """Each folded scale is the ratio-scaled scale up to one E4M3 rounding: relative error
+    <= 2**-4 (the pages' <= 6.2 %) while the result is normal (>= 2**-6), and <= half a
+    subnormal step (2**-10) below that."""
+    rng = np.random.default_rng(102)
+    sf = _rand_sf(rng, (256, 16), lo=0x01)
+    gss = [1.0, 1.82, 2.75, 7.3, 16.0]
+    outs, gs_c = oracle.fold_segments([sf] * len(gss), gss)
+    for g, o in zip(gss, outs):
+        exact = oracle.e4m3_decode(sf) * np.float64(np.float32(gs_c / np.float32(g)))
+        got = oracle.e4m3_decode(o)
+        normal = exact >= 2.0 ** -6
+        assert np.all(np.abs(got - exact)[normal] <= 2.0 ** -4 * exact[normal] + 1e-30)
+        assert np.all(np.abs(got - exact)[~normal] <= 2.0 ** -10)
+        assert np.all(got <= 448.0)
+
+
+def test_fold_dequantised_weights_within_bound():
+    """Folding changes each decoded weight by at most 2**-4 of itself (normal scales)."""
+    rng = np.random.default_rng(103)
+    segs = [rng.standard_normal((32, 64)).astype(np.float32) * m for m in (0.02, 0.1, 0.32)]
+    q = [oracle.quantize(w, oracle.global_scale(w)) + (oracle.global_scale(w),) for w in segs]
+    outs, gs_c = oracle.fold_segments([sf for _, sf, _ in q], [g for _, _, g in q])
+    for (codes, sf, g), sf2 in zip(q, outs):
+        before = oracle.dequantize(codes, sf, g)
+        after = oracle.dequantize(codes, sf2, gs_c)
+        assert np.all(np.abs(after - before) <= 2.0 ** -4 * np.abs(before) + 1e-12)
+
+
+def test_fold_repairs_the_shared_scale_mismatch():
+    """A fused GEMM run with one global scale: wrong by the scale ratios before folding,
+    close to the per-module result after it (blog section 罠①)."""
+    rng = np.random.default_rng(104)
+    x = rng.standard_normal((16, 256)).astype(np.float32)
+    ws = [rng.standard_normal((32, 256)).astype(np.float32) * m for m in (0.02, 0.0364, 0.055)]
+    gx = oracle.global_scale(x)
+    cx, sx = oracle.quantize(x, gx)
+    qs = [oracle.quantize(w, oracle.global_scale(w)) + (oracle.global_scale(w),) for w in ws]
+    codes = np.concatenate([c for c, _, _ in qs])
+    segs, n0 = [], 0
+    for _, _, g in qs:
+        segs.append((n0, n0 + 32, g))
+        n0 += 32
+    ref = oracle.linear(cx, sx, gx, codes, np.concatenate([s for _, s, _ in qs]), segs)
+    wrong = oracle.linear(cx, sx, gx, codes, np.concatenate([s for _, s, _ in qs]), [(0, 96, qs[0][2])])
+    folded, gs_c = oracle.fold_segments([s for _, s, _ in qs], [g for _, _, g in qs])
+    fixed = oracle.linear(cx, sx, gx, codes, np.concatenate(folded), [(0, 96, gs_c)])
+    err = lambda y: np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert err(wrong) > 0.2
+    assert err(fixed) < 0.05
