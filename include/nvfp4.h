@@ -250,6 +250,27 @@ NVFP4_API nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, c
                                                      nvfp4_stream_t stream);
 
 /*
+ * nvfp4_fold_segments - fused-group scale repair, in place: rewrites a packed fused
+ * weight whose modules carry their own global scales so that one global scale serves
+ * them all (the pages' own repair of the fused-module mismatch: blog section 罠①,
+ * "common global scale, ratio folded into the block scales, re-rounding <= 6.2 %").
+ *   gs_c = min over the modules of *segs[i].gs_w, written to *gs_common_out (device);
+ *   every block scale of module i becomes E4M3(fl32(dec(sf) * fl32(gs_c / gs_i)))
+ *   (nearest even); codes are unchanged.  Afterwards nvfp4_linear with the single
+ *   segment [(0, rows, gs_common_out)] approximates the per-module linear: each
+ *   decoded weight moves by at most 2^-4 of itself (normal scales).  The per-segment
+ *   alpha of nvfp4_linear needs no such repair and is exact; this entry point serves
+ *   checkpoints and kernels that can apply only one global scale per GEMM.
+ *   scales: device, nvfp4_scale_bytes(rows, cols) bytes, 16-byte aligned (rewritten).
+ *   segs/nseg: the modules as weight-row ranges covering [0, rows) in order (1..16).
+ *   gs_common_out: device float, must not be one of the segments' gs_w.
+ *   Padding bytes are left as they are.  Errors as nvfp4_linear's argument checks.
+ */
+NVFP4_API nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols,
+                                             const nvfp4_segment_t *segs, int nseg, float *gs_common_out,
+                                             nvfp4_stream_t stream);
+
+/*
  * nvfp4_get_device_status - read and clear the device status word of the current
  * device.  Kernels never spin forever: every wait on an mbarrier has an iteration
  * limit, and a wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the

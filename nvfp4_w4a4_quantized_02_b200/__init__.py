@@ -15,7 +15,7 @@ from typing import Optional, Sequence
 __all__ = [
     "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
     "linear_splitk", "linear_splitk_noalloc", "splitk_default", "splitk_workspace_bytes",
-    "NOALLOC_SCRATCH_BYTES",
+    "NOALLOC_SCRATCH_BYTES", "fold_segments",
     "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
 ]
 
@@ -54,7 +54,8 @@ class NVFP4Error(RuntimeError):
 _LIB = None
 SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
            "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
-           "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_get_device_status")
+           "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_fold_segments",
+           "nvfp4_get_device_status")
 
 
 def lib():
@@ -95,6 +96,8 @@ def lib():
                                               ctypes.POINTER(Segment), ctypes.c_int, ctypes.c_int,
                                               ctypes.POINTER(EpilogueParams), _c_vp, ctypes.c_int, _c_i64,
                                               ctypes.c_int, _c_vp]
+    L.nvfp4_fold_segments.restype = ctypes.c_int
+    L.nvfp4_fold_segments.argtypes = [_c_vp, _c_i64, _c_i64, ctypes.POINTER(Segment), ctypes.c_int, _c_vp, _c_vp]
     L.nvfp4_get_device_status.restype = ctypes.c_int
     L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     _LIB = L
@@ -296,6 +299,19 @@ def linear_splitk_noalloc(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Seq
     args, result, _keep = _linear_args(a, w, segments, epilogue, out_dtype, out, ldo, gates, gs_out, out_scales)
     _check(lib().nvfp4_linear_splitk_noalloc(*args, int(split_k), _stream(stream)), "nvfp4_linear_splitk_noalloc")
     return result
+
+
+def fold_segments(w: NVFP4Tensor, segments: Sequence, gs_out=None, stream=None):
+    """Fused-group repair in place: one global scale for all modules of ``w`` (the
+    ratios folded into its block scales).  Returns the common scale (float32 [1] device
+    tensor); afterwards ``linear(a, w, segments=[(0, w.rows, gs)])`` serves the weight."""
+    import torch
+    if gs_out is None:
+        gs_out = torch.empty(1, dtype=torch.float32, device=w.codes.device)
+    segs = (Segment * len(segments))(*[Segment(int(n0), int(n1), _ptr(g)) for n0, n1, g in segments])
+    _check(lib().nvfp4_fold_segments(_c_vp(w.scales.data_ptr()), w.rows, w.cols, segs, len(segments),
+                                     _c_vp(gs_out.data_ptr()), _stream(stream)), "nvfp4_fold_segments")
+    return gs_out
 
 
 def device_status() -> int:

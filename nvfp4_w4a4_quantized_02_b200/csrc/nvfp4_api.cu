@@ -10,6 +10,7 @@
 #include "nvfp4.h"
 #include "quantize.cuh"
 #include "gemm.cuh"
+#include "fold.cuh"
 
 using namespace nvfp4;
 
@@ -488,6 +489,40 @@ nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, const float
   float *scratch = nullptr;
   if (nvfp4_status_t st = noalloc_scratch(&scratch)) return st;
   return launch_splitk(p, A, W, split_k, scratch, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols, const nvfp4_segment_t *segs,
+                                   int nseg, float *gs_common_out, nvfp4_stream_t stream) {
+  if (!scales || !segs || !gs_common_out || rows < 1 || cols < 1) return NVFP4_ERR_INVALID_ARG;
+  if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(scales, 16) || !aligned(gs_common_out, 4)) return NVFP4_ERR_MISALIGNED;
+  FoldArgs a{};
+  int64_t expect = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (!segs[i].gs_w || !aligned(segs[i].gs_w, 4)) return NVFP4_ERR_INVALID_ARG;
+    if (segs[i].gs_w == gs_common_out) return NVFP4_ERR_INVALID_ARG;  // read while written
+    if (segs[i].n_begin != expect || segs[i].n_end <= segs[i].n_begin) return NVFP4_ERR_INVALID_ARG;
+    a.seg_begin[i] = static_cast<int>(segs[i].n_begin);
+    a.seg_end[i] = static_cast<int>(segs[i].n_end);
+    a.gs[i] = segs[i].gs_w;
+    expect = segs[i].n_end;
+  }
+  if (expect != rows) return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  a.scales = scales;
+  a.rows = rows;
+  a.kb = cols / 16;
+  a.kb_atoms = (a.kb + 3) / 4;
+  a.bytes = static_cast<int64_t>(nvfp4_scale_bytes(rows, cols));
+  a.nseg = nseg;
+  a.gs_common = gs_common_out;
+  const int64_t want = (a.bytes / 16 + kFoldThreads - 1) / kFoldThreads;
+  const int64_t cap = int64_t(dev->sms) * 8;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  fold_scales_kernel<<<grid, kFoldThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
 }
 
 nvfp4_status_t nvfp4_get_device_status(int *code) {
