@@ -32,6 +32,12 @@ R3  the linear: Y[m, n] = alpha(n) * sum_k Ahat[m, k] * What[n, k] with
 R4  epilogues in FP64: SiLU(gate) * up; beta = sigmoid; g = -exp(A_log) * softplus(a + dt_bias)
     with softplus(x) = max(x, 0) + log1p(exp(-|x|)).
 R5  re-quantising an output for the next layer first rounds it to BF16 (nearest even).
+R13 FP8 KV cache (blog section "KVキャッシュはFP8で十分？": static FP8 scales, one per
+    K and one per V tensor of each attention layer, calibrated and shipped with the
+    checkpoint): a cached value is E4M3(fl32(x / scale)), nearest even, saturating at
+    +-448, sign kept; it decodes to e4m3 * scale.  A calibrated scale is
+    fl32(amax / 448) (amax 0 gives 1).  Token t is written to cache row slots[t]; a
+    negative slot skips the token.
 R12 fused-group repair (blog section 罠①: the fused group is rewritten to a common
     global scale and the ratio is folded into the block scales, re-rounding error
     <= 6.2 %): the common scale is the smallest segment scale, gs_c = min gs_seg, so
@@ -52,7 +58,7 @@ __all__ = [
     "e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode",
     "global_scale", "quantize", "dequantize", "block_scaled_matmul", "linear",
     "silu", "sigmoid", "softplus", "silu_mul", "gdn_gates", "round_to_bf16",
-    "fold_segments",
+    "fold_segments", "e4m3_encode_signed", "fp8_scale", "kv_cache_fp8",
 ]
 
 E2M1_MAX = 6.0
@@ -272,3 +278,34 @@ def fold_segments(sf_segments, gs_segments):
         s = (e4m3_decode(sf).astype(np.float32) * ratio).astype(np.float32)
         out.append(e4m3_encode(s))
     return out, gs_c
+
+
+# ------------------------------------------------------------------ FP8 KV cache
+def e4m3_encode_signed(v) -> np.ndarray:
+    """Signed E4M3 byte: nearest finite magnitude, ties to even code, saturating at 448,
+    sign bit 7 copied from the input (so -0.0 -> 0x80)."""
+    v = np.asarray(v, dtype=np.float64)
+    if not np.all(np.isfinite(v)):
+        raise ValueError("e4m3_encode_signed: non-finite input")
+    mag = _nearest_even(np.abs(v), _E4M3_POS)
+    return (mag | (np.signbit(v).astype(np.int64) << 7)).astype(np.uint8)
+
+
+def fp8_scale(x) -> np.float32:
+    """Calibrated per-tensor FP8 scale fl32(amax|x| / 448); 1 for an all-zero tensor (R13)."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    return np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(E4M3_MAX))
+
+
+def kv_cache_fp8(x, scale, slots, num_slots, cache=None) -> np.ndarray:
+    """Write token rows of ``x [tokens, width]`` into an FP8 cache ``[num_slots, width]``
+    (uint8): row slots[t] = E4M3(fl32(x[t] / scale)); slots < 0 are skipped (R13)."""
+    x = np.asarray(x, dtype=np.float32)
+    tokens, width = x.shape
+    out = np.zeros((num_slots, width), np.uint8) if cache is None else np.array(cache, dtype=np.uint8)
+    q = e4m3_encode_signed((x / np.float32(scale)).astype(np.float32))
+    for t in range(tokens):
+        if slots[t] >= 0:
+            out[slots[t]] = q[t]
+    return out

@@ -427,3 +427,49 @@ def test_fold_repairs_the_shared_scale_mismatch():
     err = lambda y: np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert err(wrong) > 0.2
     assert err(fixed) < 0.05
+
+
+# ------------------------------------------------------------------ FP8 KV cache
+def test_e4m3_signed_encode_facts():
+    vals = oracle.e4m3_decode(np.arange(0x7F))                     # all finite magnitudes
+    assert np.array_equal(oracle.e4m3_encode_signed(vals), np.arange(0x7F))
+    assert np.array_equal(oracle.e4m3_encode_signed(-vals[1:]), np.arange(1, 0x7F) | 0x80)
+    assert oracle.e4m3_encode_signed(-0.0) == 0x80 and oracle.e4m3_encode_signed(0.0) == 0x00
+    assert oracle.e4m3_encode_signed(1e6) == 0x7E and oracle.e4m3_encode_signed(-1e6) == 0xFE
+    # ties between 1.0 (0x38) and 1.125 (0x39) go to the even code; just above goes up
+    assert oracle.e4m3_encode_signed(1.0625) == 0x38
+    assert oracle.e4m3_encode_signed(np.nextafter(1.0625, 2.0)) == 0x39
+    assert oracle.e4m3_encode_signed(-1.0625) == 0xB8
+
+
+def test_fp8_scale_and_roundtrip():
+    rng = np.random.default_rng(120)
+    x = rng.standard_normal((64, 128)).astype(np.float32) * 3
+    s = oracle.fp8_scale(x)
+    assert s == np.float32(np.max(np.abs(x)) / np.float32(448))
+    assert oracle.fp8_scale(np.zeros((2, 16))) == 1.0
+    cache = oracle.kv_cache_fp8(x, s, np.arange(64), 64)
+    back = oracle.e4m3_decode(cache & 0x7F) * np.where(cache & 0x80, -1, 1) * np.float64(s)
+    # the tensor amax maps to 448 (up to the fl32 division), every value within one E4M3
+    # rounding: relative 2**-4 in the normal range, half the subnormal step below it
+    r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert (cache[r, c] & 0x7F) == 0x7E
+    normal = np.abs(x / s) >= 2.0 ** -6
+    err = np.abs(back - x)
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]))
+    assert np.all(err[~normal] <= 2.0 ** -10 * np.float64(s))
+    # exactly representable values come back exactly
+    vals = oracle.e4m3_decode(np.arange(0x7F)).astype(np.float32)[None, :] * np.float32(0.5)
+    c2 = oracle.kv_cache_fp8(vals, np.float32(0.5), [0], 1)
+    assert np.array_equal(c2[0], np.arange(0x7F))
+
+
+def test_kv_cache_slot_scatter():
+    x = np.arange(4 * 16, dtype=np.float32).reshape(4, 16) - 20
+    cache = np.full((6, 16), 0x55, np.uint8)
+    out = oracle.kv_cache_fp8(x, np.float32(1.0), [5, -1, 0, 2], 6, cache=cache)
+    assert np.array_equal(out[5], oracle.e4m3_encode_signed(x[0]))
+    assert np.array_equal(out[0], oracle.e4m3_encode_signed(x[2]))
+    assert np.array_equal(out[2], oracle.e4m3_encode_signed(x[3]))
+    for r in (1, 3, 4):  # untouched rows (slot -1 wrote nothing)
+        assert np.all(out[r] == 0x55)
