@@ -17,6 +17,8 @@ One JSON line on stdout (rank 0).  Workloads (``--workload``):
   fused), each fed by the NVFP4 quantiser, at ``--M`` prefill tokens.
 * ``decode``: the same 496 linears for one decode step of ``--M`` (default 32)
   sequences through the split-K linear (weight-bandwidth bound).
+* ``kv``: the FP8 KV-cache write of one attention layer's K and V at ``--M`` prefill
+  tokens (static per-tensor scales, paged slots).
 
 Multi-GPU (torchrun): every rank runs the same workload on its own GPU with its own
 inputs (independent token batches, weak scaling); no collective touches the data
@@ -690,6 +692,62 @@ class HybridSweep(Workload):
         return f1 + f2, s1 + s2
 
 
+class KVCacheFP8(Workload):
+    """FP8 KV-cache write of one attention layer's prefill: K and V [M x 1024] BF16 (8 KV
+    heads x 128) into a paged cache (pages of 16 slots, shuffled) with static scales."""
+    unit = "GB/s"
+
+    def __init__(self, nv, M=32768, width=1024, seed=0):
+        import torch
+        self.nv, self.M, self.width = nv, M, width
+        self.name = f"kv_cache_fp8_m{M}_w{width}"
+        self.x = _gpu_student_t(M, width, seed, hot=4)
+        self.v = _gpu_student_t(M, width, seed + 1, hot=0)
+        self.k_scale = nv.fp8_scale(self.x)
+        self.v_scale = nv.fp8_scale(self.v)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed + 2)
+        num_slots = 2 * M
+        pages = torch.randperm(num_slots // 16, generator=g, device="cuda")
+        t = torch.arange(M, device="cuda")
+        self.slots = (pages[t // 16] * 16 + t % 16).to(torch.int64)
+        self.k_cache = torch.empty((num_slots, width), dtype=torch.uint8, device="cuda")
+        self.v_cache = torch.empty((num_slots, width), dtype=torch.uint8, device="cuda")
+        self.out = self.k_cache
+        self.bytes = 2.0 * M * width * 3 + 8.0 * M
+        self.launches_per_step = 1
+        self.l2_note = f"inputs larger than L2 (K, V {2 * M * width * 2 / 1e6:.0f} MB)"
+        self.dominant = ("kv_cache", self.bytes, "hbm", "kv_cache_fp8_kernel (K and V, slot scatter)")
+        self.phases = {"kv_cache": ("GB/s", self.bytes)}
+        torch.cuda.synchronize()
+
+    def work(self):
+        return self.bytes
+
+    def config(self):
+        return {"M": self.M, "width": self.width, "scales": "static per tensor (calibrated once)",
+                "bytes_per_element": 3, "slots": "pages of 16, shuffled"}
+
+    def plan(self, x):
+        nv = self.nv
+        return [("kv_cache", lambda: nv.kv_cache_fp8(x, self.v, self.k_scale, self.v_scale, self.slots,
+                                                    self.k_cache, self.v_cache))]
+
+    cpu_sample_note = "FP8 KV write of 64 tokens x 1024 (K and V); numpy oracle"
+
+    def cpu_sample(self):
+        import numpy as np
+        import oracle
+        import synth
+        k = synth.bf16_to_f32(synth.student_t_activations(64, 1024, seed=0, hot_channels=4))
+        v = synth.bf16_to_f32(synth.student_t_activations(64, 1024, seed=1, hot_channels=0))
+        ks, vs = oracle.fp8_scale(k), oracle.fp8_scale(v)
+        t0 = time.perf_counter()
+        oracle.kv_cache_fp8(k, ks, np.arange(64), 64)
+        oracle.kv_cache_fp8(v, vs, np.arange(64), 64)
+        return 2.0 * 64 * 1024 * 3 + 8.0 * 64, time.perf_counter() - t0
+
+
 class DecodeSweep(HybridSweep):
     """One decode step of the 496 linears for a batch of M sequences (concurrency 32 by
     default): the split-K linear streams every weight once per step from HBM, so the
@@ -741,7 +799,8 @@ class DecodeSweep(HybridSweep):
 
 
 WORKLOADS = {"mlp": MLPBlock, "quantize": QuantizeOnly, "gdn": GDNInProj, "linear": SmallLinear,
-             "sweep": HybridSweep, "decode": DecodeSweep}
+             "sweep": HybridSweep, "decode": DecodeSweep,
+             "kv": KVCacheFP8}
 
 
 def make_workload(args, nv):
@@ -1023,7 +1082,7 @@ class _CpuOnly:
         self.cpu_sample_note = cls.cpu_sample_note
         obj = object.__new__(cls)
         obj.M = args.M or {"mlp": 32768, "quantize": 32768, "gdn": 8192, "linear": 128, "sweep": 32768,
-                           "decode": 32}[args.workload]
+                           "decode": 32, "kv": 32768}[args.workload]
         obj.K = {"quantize": 5120, "gdn": 5120, "linear": 1024}.get(args.workload, 5120)
         obj.N = {"linear": 1024, "gdn": 12352}.get(args.workload, 0)
         obj.flops = 2.0 * obj.M * obj.N * obj.K
@@ -1031,7 +1090,8 @@ class _CpuOnly:
         self.name = {"mlp": f"mlp_block_m{obj.M}_h5120_i17408", "quantize": f"quantize_m{obj.M}_k5120",
                      "gdn": f"gdn_inproj_m{obj.M}_n12352_k5120", "linear": f"linear_m{obj.M}_n1024_k1024",
                      "sweep": f"hybrid_sweep_496_linears_m{obj.M}",
-                     "decode": f"decode_sweep_496_linears_m{obj.M}"}[args.workload]
+                     "decode": f"decode_sweep_496_linears_m{obj.M}",
+                     "kv": f"kv_cache_fp8_m{obj.M}_w1024"}[args.workload]
 
     def cpu_sample(self):
         return self.cls.cpu_sample(self.obj)

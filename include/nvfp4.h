@@ -55,7 +55,8 @@ typedef enum {
   NVFP4_ERR_MISALIGNED = 3,        /* a pointer or leading dimension violates alignment */
   NVFP4_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
   NVFP4_ERR_DEVICE_TIMEOUT = 5,    /* a kernel gave up a bounded wait (see nvfp4_get_device_status) */
-  NVFP4_ERR_UNSUPPORTED_DEVICE = 6 /* current device is not sm_100 */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 6, /* current device is not sm_100 */
+  NVFP4_ERR_DEVICE_INDEX = 7        /* a kernel skipped an out-of-range index (see nvfp4_get_device_status) */
 } nvfp4_status_t;
 
 /* Human-readable name of a status code (static storage). */
@@ -269,6 +270,34 @@ NVFP4_API nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, c
 NVFP4_API nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols,
                                              const nvfp4_segment_t *segs, int nseg, float *gs_common_out,
                                              nvfp4_stream_t stream);
+
+/*
+ * nvfp4_fp8_scale - calibrated per-tensor FP8 scale of a BF16 tensor:
+ *   *scale_out = fl32(max|x| / 448) (device), 1 when x is all zero.  The calibration
+ *   step of the pages' "ship KV scales" recipe (blog section "KVキャッシュはFP8で十分？":
+ *   static FP8 scales for the K and V tensors of every attention layer, computed on
+ *   calibration data and shipped with the checkpoint); the formula is this library's
+ *   reading.  Arguments and requirements as nvfp4_global_scale.
+ */
+NVFP4_API nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                         float *scale_out, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_kv_cache_fp8 - write the K and V rows of `tokens` tokens into an FP8 KV cache
+ * with static per-tensor scales (same source as nvfp4_fp8_scale):
+ *   k_cache[slots[t], c] = E4M3(fl32(k[t, c] / *k_scale)), likewise V with *v_scale;
+ *   nearest even, saturating at +-448, sign kept (a value decodes to e4m3 * scale).
+ *   k, v: device BF16 [tokens x width], row stride ld elements (ld >= width, ld % 8 == 0,
+ *   16-byte aligned); width % 16 == 0.  slots: device int64 [tokens]; a negative slot
+ *   skips the token; a slot >= num_slots is skipped and reported as
+ *   NVFP4_ERR_DEVICE_INDEX by nvfp4_get_device_status.  k_cache, v_cache: device
+ *   [num_slots x width] bytes, 16-byte aligned, owned by the caller; rows of other
+ *   slots are not touched.
+ */
+NVFP4_API nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_t tokens, int64_t width,
+                                            int64_t ld, const float *k_scale, const float *v_scale,
+                                            const int64_t *slots, uint8_t *k_cache, uint8_t *v_cache,
+                                            int64_t num_slots, nvfp4_stream_t stream);
 
 /*
  * nvfp4_get_device_status - read and clear the device status word of the current

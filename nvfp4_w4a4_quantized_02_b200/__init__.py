@@ -15,7 +15,7 @@ from typing import Optional, Sequence
 __all__ = [
     "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
     "linear_splitk", "linear_splitk_noalloc", "splitk_default", "splitk_workspace_bytes",
-    "NOALLOC_SCRATCH_BYTES", "fold_segments",
+    "NOALLOC_SCRATCH_BYTES", "fold_segments", "fp8_scale", "kv_cache_fp8",
     "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
 ]
 
@@ -55,7 +55,7 @@ _LIB = None
 SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
            "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
            "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_fold_segments",
-           "nvfp4_get_device_status")
+           "nvfp4_fp8_scale", "nvfp4_kv_cache_fp8", "nvfp4_get_device_status")
 
 
 def lib():
@@ -98,6 +98,11 @@ def lib():
                                               ctypes.c_int, _c_vp]
     L.nvfp4_fold_segments.restype = ctypes.c_int
     L.nvfp4_fold_segments.argtypes = [_c_vp, _c_i64, _c_i64, ctypes.POINTER(Segment), ctypes.c_int, _c_vp, _c_vp]
+    L.nvfp4_fp8_scale.restype = ctypes.c_int
+    L.nvfp4_fp8_scale.argtypes = [_c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp]
+    L.nvfp4_kv_cache_fp8.restype = ctypes.c_int
+    L.nvfp4_kv_cache_fp8.argtypes = [_c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
+                                     _c_i64, _c_vp]
     L.nvfp4_get_device_status.restype = ctypes.c_int
     L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     _LIB = L
@@ -312,6 +317,29 @@ def fold_segments(w: NVFP4Tensor, segments: Sequence, gs_out=None, stream=None):
     _check(lib().nvfp4_fold_segments(_c_vp(w.scales.data_ptr()), w.rows, w.cols, segs, len(segments),
                                      _c_vp(gs_out.data_ptr()), _stream(stream)), "nvfp4_fold_segments")
     return gs_out
+
+
+def fp8_scale(x, out=None, stream=None):
+    """Calibrated FP8 scale max|x| / 448 of a 2-D BF16 CUDA tensor (float32 [1] device tensor)."""
+    import torch
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_cuda
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().nvfp4_fp8_scale(_c_vp(x.data_ptr()), x.shape[0], x.shape[1], x.stride(0), _c_vp(out.data_ptr()),
+                                 _stream(stream)), "nvfp4_fp8_scale")
+    return out
+
+
+def kv_cache_fp8(k, v, k_scale, v_scale, slots, k_cache, v_cache, stream=None):
+    """Write K / V token rows (BF16 [tokens, width]) into FP8 caches ([num_slots, width]
+    uint8) at ``slots`` (int64 [tokens], negative = skip) with static scales."""
+    import torch
+    assert k.shape == v.shape and k.stride() == v.stride() and k.dtype == torch.bfloat16
+    assert slots.dtype == torch.int64 and k_cache.shape == v_cache.shape
+    _check(lib().nvfp4_kv_cache_fp8(_c_vp(k.data_ptr()), _c_vp(v.data_ptr()), k.shape[0], k.shape[1], k.stride(0),
+                                    _c_vp(k_scale.data_ptr()), _c_vp(v_scale.data_ptr()), _c_vp(slots.data_ptr()),
+                                    _c_vp(k_cache.data_ptr()), _c_vp(v_cache.data_ptr()), k_cache.shape[0],
+                                    _stream(stream)), "nvfp4_kv_cache_fp8")
 
 
 def device_status() -> int:

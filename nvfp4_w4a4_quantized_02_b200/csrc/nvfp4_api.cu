@@ -11,6 +11,7 @@
 #include "quantize.cuh"
 #include "gemm.cuh"
 #include "fold.cuh"
+#include "kvcache.cuh"
 
 using namespace nvfp4;
 
@@ -329,6 +330,7 @@ const char *nvfp4_status_string(int s) {
     case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
     case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
     case NVFP4_ERR_UNSUPPORTED_DEVICE: return "NVFP4_ERR_UNSUPPORTED_DEVICE";
+    case NVFP4_ERR_DEVICE_INDEX: return "NVFP4_ERR_DEVICE_INDEX";
     default: return "NVFP4_ERR_UNKNOWN";
   }
 }
@@ -522,6 +524,61 @@ nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols, 
   const int64_t cap = int64_t(dev->sms) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
   fold_scales_kernel<<<grid, kFoldThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
+nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *scale_out,
+                               nvfp4_stream_t stream) {
+  if (!x_bf16 || !scale_out || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x_bf16, 16) || ld % 8 != 0 || !aligned(scale_out, 4)) return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scale_out, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  AmaxArgs a;
+  a.x = static_cast<const uint16_t *>(x_bf16);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.amax_bits = reinterpret_cast<unsigned int *>(scale_out);
+  const int64_t vecs = rows * (cols / 8);
+  const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
+  const int64_t cap = int64_t(dev->sms) * 8;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
+  amax_kernel<<<grid, kAmaxThreads, 0, s>>>(a);
+  fp8_scale_finalize_kernel<<<1, 1, 0, s>>>(scale_out);
+  return launch_status();
+}
+
+nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_t tokens, int64_t width,
+                                  int64_t ld, const float *k_scale, const float *v_scale, const int64_t *slots,
+                                  uint8_t *k_cache, uint8_t *v_cache, int64_t num_slots, nvfp4_stream_t stream) {
+  if (!k_bf16 || !v_bf16 || !k_scale || !v_scale || !slots || !k_cache || !v_cache) return NVFP4_ERR_INVALID_ARG;
+  if (tokens < 1 || width < 1 || ld < width || num_slots < 1) return NVFP4_ERR_INVALID_ARG;
+  if (width % 16 != 0 || tokens > kMaxDim || width > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(k_bf16, 16) || !aligned(v_bf16, 16) || ld % 8 != 0 || !aligned(k_scale, 4) ||
+      !aligned(v_scale, 4) || !aligned(slots, 8) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  KvArgs a;
+  a.k = static_cast<const uint16_t *>(k_bf16);
+  a.v = static_cast<const uint16_t *>(v_bf16);
+  a.tokens = tokens;
+  a.width = width;
+  a.ld = ld;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.slots = slots;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.num_slots = num_slots;
+  const int64_t chunks = 2 * tokens * (width / 16);
+  const int64_t want = (chunks + kKvThreads - 1) / kKvThreads;
+  const int64_t cap = int64_t(dev->sms) * 16;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  kv_cache_fp8_kernel<<<grid, kKvThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launch_status();
 }
 

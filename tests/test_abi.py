@@ -46,8 +46,9 @@ def test_scale_bytes_matches_layout_reading(L):
 
 
 def test_status_strings(L):
-    names = [L.nvfp4_status_string(i).decode() for i in range(7)]
+    names = [L.nvfp4_status_string(i).decode() for i in range(8)]
     assert names[0] == "NVFP4_OK" and names[5] == "NVFP4_ERR_DEVICE_TIMEOUT"
+    assert names[7] == "NVFP4_ERR_DEVICE_INDEX"
     assert L.nvfp4_status_string(99).decode() == "NVFP4_ERR_UNKNOWN"
 
 
