@@ -493,6 +493,30 @@ class GDNInProj(Workload):
                                        out_dtype="bf16", out=self.out)),
         ]
 
+    def extra(self, torch):
+        """The pages' offline repair of the same fused weight (nvfp4_fold_segments on a copy of
+        its scale buffer), timed separately: a pass over the 3.9 MB scale buffer."""
+        nv = self.nv
+        w = nv.NVFP4Tensor(self.w.codes, self.w.scales.clone(), self.w.gs, self.w.rows, self.w.cols)
+        gs_c = torch.empty(1, dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            w.scales.copy_(self.w.scales)
+            nv.fold_segments(w, self.segs, gs_out=gs_c)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 20
+        ms = 0.0
+        for _ in range(n):
+            w.scales.copy_(self.w.scales)
+            s.record()
+            nv.fold_segments(w, self.segs, gs_out=gs_c)
+            e.record()
+            torch.cuda.synchronize()
+            ms += s.elapsed_time(e)
+        ms /= n
+        b = 2.0 * w.scales.numel()
+        return {"fold_segments": {"ms": round(ms, 5), "GB/s": round(b / ms / 1e6, 1), "bytes": b}}
+
     cpu_sample_note = ("GDN in-proj sample: 32 token rows x 320 weight rows (64 each of q/k/v/z + 32 beta + "
                        "32 alpha), K=5120; quantise X + fused linear + gates; numpy FP64 oracle")
 

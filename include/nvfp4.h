@@ -285,8 +285,9 @@ NVFP4_API nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64
 /*
  * nvfp4_kv_cache_fp8 - write the K and V rows of `tokens` tokens into an FP8 KV cache
  * with static per-tensor scales (same source as nvfp4_fp8_scale):
- *   k_cache[slots[t], c] = E4M3(fl32(k[t, c] / *k_scale)), likewise V with *v_scale;
- *   nearest even, saturating at +-448, sign kept (a value decodes to e4m3 * scale).
+ *   k_cache[slots[t], c] = E4M3(fl32(k[t, c] * fl32(1 / *k_scale))), likewise V with
+ *   *v_scale; nearest even, saturating at +-448, sign kept (a value decodes to
+ *   e4m3 * scale).
  *   k, v: device BF16 [tokens x width], row stride ld elements (ld >= width, ld % 8 == 0,
  *   16-byte aligned); width % 16 == 0.  slots: device int64 [tokens]; a negative slot
  *   skips the token; a slot >= num_slots is skipped and reported as

@@ -1,9 +1,10 @@
 // FP8 KV cache with static per-tensor scales (blog "27BハイブリッドLLMを4ビットで動かす",
 // section "KVキャッシュはFP8で十分？": the attention layers' K and V tensors are cached in
 // FP8 with calibrated scales shipped in the checkpoint).  Each token row of K and V is
-// written to its cache slot as E4M3(fl32(x / scale)) (nearest even, saturating at +-448,
-// sign kept); a negative slot skips the token.  HBM-bound: 2 bytes read and 1 written
-// per element.
+// written to its cache slot as E4M3(fl32(x * fl32(1 / scale))) (nearest even,
+// saturating at +-448, sign kept); a negative slot skips the token.  HBM-bound: 2 bytes
+// read and 1 written per element.  A thread handles one 16-element chunk of a token
+// row in K and the same chunk in V (one slot read for both).
 #pragma once
 
 #include "quant_math.cuh"
@@ -22,37 +23,46 @@ struct KvArgs {
   int64_t num_slots;
 };
 
+// 16 BF16 values (two 16-byte words) -> 16 E4M3 bytes of x * inv.
+__device__ __forceinline__ uint4 fp8_chunk(const uint4 &w0, const uint4 &w1, float inv) {
+  const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float x0 = __fmul_rn(__uint_as_float(w[2 * j] << 16), inv);
+    const float x1 = __fmul_rn(__uint_as_float(w[2 * j] & 0xFFFF0000u), inv);
+    const float x2 = __fmul_rn(__uint_as_float(w[2 * j + 1] << 16), inv);
+    const float x3 = __fmul_rn(__uint_as_float(w[2 * j + 1] & 0xFFFF0000u), inv);
+    out[j] = static_cast<uint32_t>(cvt_e4m3x2(x1, x0)) | (static_cast<uint32_t>(cvt_e4m3x2(x3, x2)) << 16);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 __global__ void __launch_bounds__(kKvThreads) kv_cache_fp8_kernel(const __grid_constant__ KvArgs a) {
-  const float ks = __ldg(a.k_scale), vs = __ldg(a.v_scale);
-  const int64_t per_row = a.width / 16;
-  const int64_t n = a.tokens * per_row;  // 16-element chunks per tensor
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < 2 * n;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const bool is_v = idx >= n;
-    const int64_t i = is_v ? idx - n : idx;
-    const int64_t t = i / per_row;
-    const int64_t c = (i - t * per_row) * 16;
+  const float k_inv = __frcp_rn(__ldg(a.k_scale)), v_inv = __frcp_rn(__ldg(a.v_scale));
+  const int64_t per_row = a.width / 16;  // 16-element chunks per row
+  // chunk idx = token * per_row + column chunk: shifts when per_row is a power of two
+  const bool pow2 = (per_row & (per_row - 1)) == 0;
+  const int shift = __ffsll(per_row) - 1;
+  const int64_t total = (int64_t)gridDim.x * kKvThreads;
+  const int64_t n = a.tokens * per_row;
+  for (int64_t idx = (int64_t)blockIdx.x * kKvThreads + threadIdx.x; idx < n; idx += total) {
+    const int64_t t = pow2 ? idx >> shift : idx / per_row;
+    const int64_t cc = idx - t * per_row;
+    if (t >= a.tokens) continue;
     const int64_t slot = __ldg(a.slots + t);
     if (slot < 0) continue;
     if (slot >= a.num_slots) {  // never write outside the cache; report it
       atomicCAS(&g_device_status, 0, kStatusBadIndex);
       continue;
     }
-    const uint4 *src = reinterpret_cast<const uint4 *>((is_v ? a.v : a.k) + t * a.ld + c);
-    const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
-    const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    const float s = is_v ? vs : ks;
-    uint32_t out[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float x0 = __fdiv_rn(__uint_as_float(w[2 * j] << 16), s);
-      const float x1 = __fdiv_rn(__uint_as_float(w[2 * j] & 0xFFFF0000u), s);
-      const float x2 = __fdiv_rn(__uint_as_float(w[2 * j + 1] << 16), s);
-      const float x3 = __fdiv_rn(__uint_as_float(w[2 * j + 1] & 0xFFFF0000u), s);
-      out[j] = static_cast<uint32_t>(cvt_e4m3x2(x1, x0)) | (static_cast<uint32_t>(cvt_e4m3x2(x3, x2)) << 16);
-    }
-    uint8_t *dst = (is_v ? a.v_cache : a.k_cache) + slot * a.width + c;
-    *reinterpret_cast<uint4 *>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+    const int64_t off = t * a.ld + cc * 16;
+    const uint4 *ks = reinterpret_cast<const uint4 *>(a.k + off);
+    const uint4 *vs = reinterpret_cast<const uint4 *>(a.v + off);
+    const uint4 k0 = __ldcs(ks), k1 = __ldcs(ks + 1), v0 = __ldcs(vs), v1 = __ldcs(vs + 1);
+    const int64_t dst = slot * a.width + cc * 16;
+    *reinterpret_cast<uint4 *>(a.k_cache + dst) = fp8_chunk(k0, k1, k_inv);
+    *reinterpret_cast<uint4 *>(a.v_cache + dst) = fp8_chunk(v0, v1, v_inv);
   }
 }
 

@@ -34,7 +34,8 @@ R4  epilogues in FP64: SiLU(gate) * up; beta = sigmoid; g = -exp(A_log) * softpl
 R5  re-quantising an output for the next layer first rounds it to BF16 (nearest even).
 R13 FP8 KV cache (blog section "KVキャッシュはFP8で十分？": static FP8 scales, one per
     K and one per V tensor of each attention layer, calibrated and shipped with the
-    checkpoint): a cached value is E4M3(fl32(x / scale)), nearest even, saturating at
+    checkpoint): the reciprocal of the shipped scale is taken once, inv = fl32(1 /
+    scale), and a cached value is E4M3(fl32(x * inv)), nearest even, saturating at
     +-448, sign kept; it decodes to e4m3 * scale.  A calibrated scale is
     fl32(amax / 448) (amax 0 gives 1).  Token t is written to cache row slots[t]; a
     negative slot skips the token.
@@ -300,11 +301,12 @@ def fp8_scale(x) -> np.float32:
 
 def kv_cache_fp8(x, scale, slots, num_slots, cache=None) -> np.ndarray:
     """Write token rows of ``x [tokens, width]`` into an FP8 cache ``[num_slots, width]``
-    (uint8): row slots[t] = E4M3(fl32(x[t] / scale)); slots < 0 are skipped (R13)."""
+    (uint8): row slots[t] = E4M3(fl32(x[t] * fl32(1 / scale))); slots < 0 are skipped (R13)."""
     x = np.asarray(x, dtype=np.float32)
     tokens, width = x.shape
     out = np.zeros((num_slots, width), np.uint8) if cache is None else np.array(cache, dtype=np.uint8)
-    q = e4m3_encode_signed((x / np.float32(scale)).astype(np.float32))
+    inv = np.float32(np.float32(1.0) / np.float32(scale))
+    q = e4m3_encode_signed((x * inv).astype(np.float32))
     for t in range(tokens):
         if slots[t] >= 0:
             out[slots[t]] = q[t]

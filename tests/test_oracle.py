@@ -458,10 +458,11 @@ def test_fp8_scale_and_roundtrip():
     err = np.abs(back - x)
     assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]))
     assert np.all(err[~normal] <= 2.0 ** -10 * np.float64(s))
-    # exactly representable values come back exactly
+    # exactly representable values come back exactly (power-of-two scale: exact reciprocal)
     vals = oracle.e4m3_decode(np.arange(0x7F)).astype(np.float32)[None, :] * np.float32(0.5)
     c2 = oracle.kv_cache_fp8(vals, np.float32(0.5), [0], 1)
     assert np.array_equal(c2[0], np.arange(0x7F))
+
 
 
 def test_kv_cache_slot_scatter():
