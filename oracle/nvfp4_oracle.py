@@ -44,6 +44,13 @@ R12 fused-group repair (blog section 罠①: the fused group is rewritten to a c
     <= 6.2 %): the common scale is the smallest segment scale, gs_c = min gs_seg, so
     every ratio is <= 1 and no block scale saturates; each block scale becomes
     sf' = E4M3(fl32(dec(sf) * fl32(gs_c / gs_seg))), nearest even; codes are kept.
+R14 GDN recurrence (blog section "Gated DeltaNetの仕組み"): per value head, a state
+    S in R^{d_k x d_v} evolves as S_t = alpha_t S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T
+    with alpha_t = exp(g_t), g and beta the gate outputs of the in-projection's
+    epilogue (R4).  The pages give no read-out: o_t = S_t^T q_t (the state read with the
+    query, after the update).  q and k are taken as given (the model's short
+    convolution and normalisation are neither linears nor on the pages); value head h
+    reads key head h // (H_v / H_k).
 
 Float32 steps (R1, R2) use numpy float32 scalars/arrays, whose +, *, / are IEEE-754
 single precision, round to nearest even: the same operations a correct kernel
@@ -59,7 +66,7 @@ __all__ = [
     "e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode",
     "global_scale", "quantize", "dequantize", "block_scaled_matmul", "linear",
     "silu", "sigmoid", "softplus", "silu_mul", "gdn_gates", "round_to_bf16",
-    "fold_segments", "e4m3_encode_signed", "fp8_scale", "kv_cache_fp8",
+    "fold_segments", "e4m3_encode_signed", "fp8_scale", "kv_cache_fp8", "gdn_recurrence",
 ]
 
 E2M1_MAX = 6.0
@@ -311,3 +318,33 @@ def kv_cache_fp8(x, scale, slots, num_slots, cache=None) -> np.ndarray:
         if slots[t] >= 0:
             out[slots[t]] = q[t]
     return out
+
+
+# ---------------------------------------------------------------- GDN recurrence
+def gdn_recurrence(q, k, v, g, beta, state=None):
+    """Gated delta-rule recurrence of one sequence, in FP64 (reading R14).
+
+    q, k: [T, H_k, d_k]; v: [T, H_v, d_v]; g, beta: [T, H_v]; state: [H_v, d_k, d_v] or
+    None (zeros).  Returns (o [T, H_v, d_v], final state).  Token by token, as written:
+    S <- exp(g) S + beta k (v - S^T k)^T ;  o = S^T q.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    g = np.asarray(g, np.float64)
+    beta = np.asarray(beta, np.float64)
+    T, hk, dk = k.shape
+    hv, dv = v.shape[1], v.shape[2]
+    if hv % hk:
+        raise ValueError("value heads must be a multiple of key heads")
+    rep = hv // hk
+    S = np.zeros((hv, dk, dv)) if state is None else np.array(state, np.float64)
+    o = np.empty((T, hv, dv))
+    for t in range(T):
+        kt = np.repeat(k[t], rep, axis=0)                  # [H_v, d_k]
+        qt = np.repeat(q[t], rep, axis=0)
+        pred = np.einsum("hij,hi->hj", S, kt)              # S^T k
+        upd = beta[t][:, None] * (v[t] - pred)             # beta (v - S^T k)
+        S = np.exp(g[t])[:, None, None] * S + kt[:, :, None] * upd[:, None, :]
+        o[t] = np.einsum("hij,hi->hj", S, qt)              # S^T q
+    return o, S

@@ -474,3 +474,68 @@ def test_kv_cache_slot_scatter():
     assert np.array_equal(out[2], oracle.e4m3_encode_signed(x[3]))
     for r in (1, 3, 4):  # untouched rows (slot -1 wrote nothing)
         assert np.all(out[r] == 0x55)
+
+
+# ---------------------------------------------------------------- GDN recurrence
+def _unit(rng, shape):
+    x = rng.standard_normal(shape)
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def test_gdn_no_write_no_decay_keeps_state():
+    rng = np.random.default_rng(140)
+    T, hk, hv, d = 5, 2, 4, 8
+    q, k = _unit(rng, (T, hk, d)), _unit(rng, (T, hk, d))
+    v = rng.standard_normal((T, hv, d))
+    S0 = rng.standard_normal((hv, d, d))
+    o, S = oracle.gdn_recurrence(q, k, v, np.zeros((T, hv)), np.zeros((T, hv)), S0)
+    assert np.array_equal(S, S0)
+    qq = np.repeat(q, 2, axis=1)
+    assert np.allclose(o, np.einsum("hij,thi->thj", S0, qq), rtol=1e-14, atol=1e-14)
+    # pure decay: beta = 0 scales the state by prod(alpha)
+    g = -rng.uniform(0, 0.1, (T, hv))
+    _, S2 = oracle.gdn_recurrence(q, k, v, g, np.zeros((T, hv)), S0)
+    assert np.allclose(S2, np.exp(g.sum(0))[:, None, None] * S0, rtol=1e-13)
+
+
+def test_gdn_delta_rule_overwrites_along_the_key():
+    """alpha = 1, beta = 1, |k| = 1: after a write the state maps k_t exactly to v_t
+    (the write replaces what the state predicted along k_t; blog mechanism ③)."""
+    rng = np.random.default_rng(141)
+    T, hk, hv, d = 6, 1, 2, 16
+    q, k = _unit(rng, (T, hk, d)), _unit(rng, (T, hk, d))
+    v = rng.standard_normal((T, hv, d))
+    S0 = rng.standard_normal((hv, d, d))
+    for t in range(1, T + 1):
+        _, S = oracle.gdn_recurrence(q[:t], k[:t], v[:t], np.zeros((t, hv)), np.ones((t, hv)), S0)
+        assert np.allclose(np.einsum("hij,i->hj", S, k[t - 1, 0]), v[t - 1], rtol=1e-12, atol=1e-12)
+    # and directions orthogonal to k_t are left as they were
+    _, S1 = oracle.gdn_recurrence(q[:1], k[:1], v[:1], np.zeros((1, hv)), np.ones((1, hv)), S0)
+    w = rng.standard_normal(d)
+    w -= (w @ k[0, 0]) * k[0, 0]
+    assert np.allclose(np.einsum("hij,i->hj", S1, w), np.einsum("hij,i->hj", S0, w), atol=1e-12)
+
+
+def test_gdn_single_step_by_hand():
+    """d = 2, one head: S0 = [[1, 2], [3, 4]], k = (1, 0), v = (10, 20), alpha = 0.5,
+    beta = 0.25, q = (0, 1).  S0^T k = (1, 2); beta (v - S0^T k) = (2.25, 4.5);
+    S1 = 0.5 S0 + k (2.25, 4.5) = [[2.75, 5.5], [1.5, 2]]; o = S1^T q = (1.5, 2)."""
+    S0 = np.array([[[1.0, 2.0], [3.0, 4.0]]])
+    o, S = oracle.gdn_recurrence(np.array([[[0.0, 1.0]]]), np.array([[[1.0, 0.0]]]),
+                                 np.array([[[10.0, 20.0]]]), np.log([[0.5]]), np.array([[0.25]]), S0)
+    assert np.allclose(S[0], [[2.75, 5.5], [1.5, 2.0]], rtol=1e-15)
+    assert np.allclose(o[0, 0], [1.5, 2.0], rtol=1e-15)
+
+
+def test_gdn_linear_in_values_from_zero_state():
+    rng = np.random.default_rng(142)
+    T, hk, hv, d = 7, 2, 4, 8
+    q, k = _unit(rng, (T, hk, d)), _unit(rng, (T, hk, d))
+    v = rng.standard_normal((T, hv, d))
+    g, b = -rng.uniform(0, 2, (T, hv)), rng.uniform(0, 1, (T, hv))
+    o1, _ = oracle.gdn_recurrence(q, k, v, g, b)
+    o2, _ = oracle.gdn_recurrence(q, k, 3.0 * v, g, b)
+    assert np.allclose(o2, 3.0 * o1, rtol=1e-12, atol=1e-12)
+    # value head h reads key head h // 2
+    o3, _ = oracle.gdn_recurrence(q[:, :1], k[:, :1], v[:, :2], g[:, :2], b[:, :2])
+    assert np.allclose(o3, o1[:, :2], rtol=1e-13)
