@@ -19,6 +19,11 @@ One JSON line on stdout (rank 0).  Workloads (``--workload``):
   sequences through the split-K linear (weight-bandwidth bound).
 * ``kv``: the FP8 KV-cache write of one attention layer's K and V at ``--M`` prefill
   tokens (static per-tensor scales, paged slots).
+* ``gdn_rec``: the gated delta-rule recurrence of one GDN layer over ``--M`` prefill
+  tokens (sequences of 4096; 16 key / 32 value heads of 128, FP32 state), consuming
+  q|k|v rows and the gate epilogue's g / beta; FP32-ALU bound.
+* ``gdn_decode``: one decode step of that recurrence for ``--M`` (default 32)
+  sequences over their carried states; bound by the state's HBM traffic.
 
 Multi-GPU (torchrun): every rank runs the same workload on its own GPU with its own
 inputs (independent token batches, weak scaling); no collective touches the data
@@ -45,6 +50,8 @@ sys.path.insert(0, ROOT)
 METRIC = "NVFP4 W4A4 linear TFLOPS & % of B200 dense FP4 peak; quantise GB/s vs HBM"
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP32_LANES_PER_SM = 128     # FP32 FMA lanes per SM (4 sub-partitions x 32)
+SM_MAX_MHZ = 1965.0         # clocks.max.sm of the B200
 L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
 
 
@@ -283,6 +290,30 @@ def _gdn_gate_tensors(torch, M, seed):
                 beta_out=beta, g_out=gate)
 
 
+def _gpu_gdn_rec_inputs(M, seq_len, seed, hk=16, hv=32, d=128):
+    """GDN recurrence inputs on the device, same recipe as ``synth.gdn_recurrence_inputs``
+    (unit-norm q / k heads in BF16, v ~ N(0,1) BF16, g = -c_h U(0.5, 1.5) with c_h
+    log-uniform in [2e-5, 0.5], beta ~ U(0.05, 1)), drawn with torch's generator.
+    Rows are q | k | v (width 2 hk d + hv d)."""
+    import math
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    wk, wv = hk * d, hv * d
+    rows = torch.empty((M, 2 * wk + wv), dtype=torch.bfloat16, device="cuda")
+    for c in (0, wk):
+        x = torch.randn((M, hk, d), generator=g, device="cuda")
+        rows[:, c:c + wk] = (x / x.norm(dim=-1, keepdim=True)).reshape(M, wk).to(torch.bfloat16)
+    rows[:, 2 * wk:] = torch.randn((M, wv), generator=g, device="cuda").to(torch.bfloat16)
+    lo, hi = math.log(2e-5), math.log(0.5)
+    rate = torch.exp(lo + (hi - lo) * torch.rand(hv, generator=g, device="cuda"))
+    gate = -rate[None, :] * (0.5 + torch.rand((M, hv), generator=g, device="cuda"))
+    beta = 0.05 + 0.95 * torch.rand((M, hv), generator=g, device="cuda")
+    n = (M + seq_len - 1) // seq_len
+    cu = torch.tensor([min(i * seq_len, M) for i in range(n + 1)], dtype=torch.int32, device="cuda")
+    return rows, gate.contiguous(), beta.contiguous(), cu
+
+
 # --------------------------------------------------------------- workloads
 class Workload:
     """Inputs resident on the device plus a ``step(tm)`` that runs the hot path once.
@@ -310,6 +341,7 @@ class Workload:
 
     cpu_sample_note = ""
     use_graph = False  # replay the step as a CUDA graph (launch-bound workloads)
+    dtype = None       # arithmetic type label (default: by unit)
 
     def plan(self, x):
         """The step as a list of (phase, launch) pairs; every launch writes preallocated buffers."""
@@ -822,9 +854,113 @@ class DecodeSweep(HybridSweep):
                                 "weight_GB/s": round(self.packed_bytes / ms_step / 1e6, 1)}}
 
 
+class GDNRecurrence(Workload):
+    """Gated delta-rule recurrence of one GDN layer at M prefill tokens (sequences of
+    4096, fresh states): 16 key / 32 value heads of 128, q|k|v BF16 rows, g / beta FP32
+    [M x 32] as the gate epilogue writes them, FP32 state, BF16 output [M x 4096].
+    Algorithmic FLOPs per token and value head: 7 d_k d_v (prediction S^T k 2, decay 1,
+    rank-1 write 2, read-out S^T q 2)."""
+    unit = "TFLOP/s"
+    dtype = "fp32 state and arithmetic (bf16 q/k/v/out)"
+    SEQ = 4096
+
+    def __init__(self, nv, M=8192, seed=0):
+        import torch
+        self.nv, self.M = nv, M
+        self.n_seqs = (M + self.SEQ - 1) // self.SEQ
+        self.name = f"gdn_recurrence_t{M}_seq{min(M, self.SEQ)}_hk16_hv32_d128"
+        self.x, self.g, self.beta, self.cu = _gpu_gdn_rec_inputs(M, self.SEQ, seed)
+        self.state = torch.zeros((self.n_seqs, 32, 128, 128), dtype=torch.float32, device="cuda")
+        self.out = torch.empty((M, 32 * 128), dtype=torch.bfloat16, device="cuda")
+        self.flops = 7.0 * 128 * 128 * 32 * M
+        self.launches_per_step = 1
+        self.l2_note = (f"inputs larger than L2 (q|k|v rows {M * 8192 * 2 / 1e6:.0f} MB, out "
+                        f"{M * 4096 * 2 / 1e6:.0f} MB)")
+        self.dominant = ("gdn_recurrence", self.flops, "alu", "gdn recurrence_kernel<32> (state in registers)")
+        self.phases = {"gdn_recurrence": ("ALU", self.flops)}
+        torch.cuda.synchronize()
+
+    def work(self):
+        return self.flops
+
+    def config(self):
+        return {"tokens": self.M, "seq_len": min(self.M, self.SEQ), "n_seqs": self.n_seqs, "key_heads": 16,
+                "value_heads": 32, "head_dim": 128, "state": "fp32, fresh per sequence",
+                "flops_per_token_head": "7 * 128 * 128"}
+
+    def plan(self, x):
+        nv = self.nv
+        q, k, v = x[:, :2048], x[:, 2048:4096], x[:, 4096:]
+        return [("gdn_recurrence", lambda: nv.gdn_recurrence(q, k, v, self.g, self.beta, self.cu, self.state,
+                                                            initial_state=False, out=self.out))]
+
+    cpu_sample_note = "GDN recurrence, 1 sequence x 64 tokens x 4 value heads; numpy oracle (fp64)"
+
+    def cpu_sample(self):
+        import oracle
+        import synth
+        d = synth.gdn_recurrence_inputs([64], 2, 4, seed=0)
+        f = lambda c, h: synth.bf16_to_f32(d["rows"][:, c:c + h * 128]).reshape(64, h, 128)
+        q, k, v = f(d["q_col"], 2), f(d["k_col"], 2), f(d["v_col"], 4)
+        t0 = time.perf_counter()
+        oracle.gdn_recurrence(q, k, v, d["g"], d["beta"])
+        return 7.0 * 128 * 128 * 4 * 64, time.perf_counter() - t0
+
+
+class GDNDecode(GDNRecurrence):
+    """One decode step of the GDN recurrence for M sequences (one token each) over their
+    carried FP32 states [M x 32 x 128 x 128]: every state is read and written once, so
+    the bound is HBM bandwidth.  Algorithmic bytes: state 2 x 64 KiB per (sequence, value
+    head), q|k|v 16 KiB, g / beta 256 B and BF16 output 8 KiB per sequence."""
+    unit = "GB/s"
+    SEQ = 1
+    use_graph = True  # a ~20 us step: replay it as a graph so host launch gaps do not count
+
+    def __init__(self, nv, M=32, seed=0):
+        import torch
+        super().__init__(nv, M=M, seed=seed)
+        self.name = f"gdn_decode_b{M}_hk16_hv32_d128"
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed + 1)
+        self.state.copy_(0.3 * torch.randn(self.state.shape, generator=g, device="cuda"))
+        self.bytes = M * (32 * 2 * 128 * 128 * 4 + 8192 * 2 + 2 * 32 * 4 + 4096 * 2) + 4.0 * (M + 1)
+        self.l2_note = f"states {self.state.numel() * 4 / 1e6:.0f} MB read and written per step (> L2)"
+        self.dominant = ("gdn_recurrence", self.bytes, "hbm", "gdn recurrence_kernel<8> (state read + write)")
+        self.phases = {"gdn_recurrence": ("GB/s", self.bytes)}
+
+    def work(self):
+        return self.bytes
+
+    def config(self):
+        return {"sequences": self.M, "tokens_per_sequence": 1, "key_heads": 16, "value_heads": 32,
+                "head_dim": 128, "state": "fp32, carried (read and written each step)"}
+
+    def plan(self, x):
+        nv = self.nv
+        q, k, v = x[:, :2048], x[:, 2048:4096], x[:, 4096:]
+        return [("gdn_recurrence", lambda: nv.gdn_recurrence(q, k, v, self.g, self.beta, self.cu, self.state,
+                                                            initial_state=True, out=self.out))]
+
+    cpu_sample_note = "GDN decode step, 8 sequences x 32 value heads; numpy oracle (fp64)"
+
+    def cpu_sample(self):
+        import numpy as np
+        import oracle
+        import synth
+        d = synth.gdn_recurrence_inputs([1] * 8, 16, 32, seed=0)
+        f = lambda c, h: synth.bf16_to_f32(d["rows"][:, c:c + h * 128]).reshape(8, h, 128)
+        q, k, v = f(d["q_col"], 16), f(d["k_col"], 16), f(d["v_col"], 32)
+        S0 = np.random.default_rng(0).standard_normal((8, 32, 128, 128)) * 0.3
+        t0 = time.perf_counter()
+        for s in range(8):
+            oracle.gdn_recurrence(q[s:s + 1], k[s:s + 1], v[s:s + 1], d["g"][s:s + 1], d["beta"][s:s + 1], S0[s])
+        per_seq = 32 * 2 * 128 * 128 * 4 + 8192 * 2 + 2 * 32 * 4 + 4096 * 2
+        return 8.0 * per_seq, time.perf_counter() - t0
+
+
 WORKLOADS = {"mlp": MLPBlock, "quantize": QuantizeOnly, "gdn": GDNInProj, "linear": SmallLinear,
              "sweep": HybridSweep, "decode": DecodeSweep,
-             "kv": KVCacheFP8}
+             "kv": KVCacheFP8, "gdn_rec": GDNRecurrence, "gdn_decode": GDNDecode}
 
 
 def make_workload(args, nv):
@@ -932,6 +1068,9 @@ def run_ours(args, ws, rank):
     else:
         for key, d in tm.summary().items():
             per_phase[key] = {"launches": d["launches"] // args.steps, "ms_step": d["ms_total"] / args.steps}
+    # FP32 FMA peak of the device: SMs x lanes x 2 FLOP x max SM clock (sampled max, else nominal)
+    sm_max = (clocks or {}).get("sm_max_mhz") or SM_MAX_MHZ
+    alu_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
     kernels = {}
     for key, (unit, amount) in wl.phases.items():
         if key not in per_phase:
@@ -941,6 +1080,9 @@ def run_ours(args, ws, rank):
         if unit == "GB/s":
             d["GB/s"] = round(amount / ms / 1e6, 1)
             d["frac_hbm"] = round(d["GB/s"] / peaks["hbm_gbs"], 4)
+        elif unit == "ALU":
+            d["TFLOP/s"] = round(amount / ms / 1e9, 2)
+            d["frac_fp32_peak"] = round(d["TFLOP/s"] / alu_peak, 4)
         else:
             d["TFLOP/s"] = round(amount / ms / 1e9, 1)
             d["frac_fp4_peak"] = round(d["TFLOP/s"] / (peaks["bf16_tflops_sustained"] * FP4_OVER_BF16), 4)
@@ -952,6 +1094,11 @@ def run_ours(args, ws, rank):
         achieved = per_launch / avg_ms / 1e6
         peak, unit = peaks["hbm_gbs"], "GB/s"
         note = f"{peak_src} hbm_gbs (copy bandwidth)"
+    elif bound == "alu":
+        achieved = per_launch / avg_ms / 1e9
+        peak, unit = round(alu_peak, 2), "TFLOP/s"
+        note = (f"derived FP32 FMA peak: {props.multi_processor_count} SMs x {FP32_LANES_PER_SM} lanes x 2 FLOP x "
+                f"{sm_max:.0f} MHz")
     else:
         achieved = per_launch / avg_ms / 1e9
         peak, unit = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16, "TFLOP/s"
@@ -973,7 +1120,8 @@ def run_ours(args, ws, rank):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "nvfp4(e2m1+e4m3)->fp32 acc" if wl.unit != "GB/s" else "bf16->nvfp4",
+        "vs_baseline": None,
+        "dtype": wl.dtype or ("nvfp4(e2m1+e4m3)->fp32 acc" if wl.unit != "GB/s" else "bf16->nvfp4"),
         "data": "synthetic", "config": cfg, "roofline": roof, "kernels": kernels, "e2e": e2e,
         "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks, "peaks_source": peak_src,
     }
@@ -1106,7 +1254,7 @@ class _CpuOnly:
         self.cpu_sample_note = cls.cpu_sample_note
         obj = object.__new__(cls)
         obj.M = args.M or {"mlp": 32768, "quantize": 32768, "gdn": 8192, "linear": 128, "sweep": 32768,
-                           "decode": 32, "kv": 32768}[args.workload]
+                           "decode": 32, "kv": 32768, "gdn_rec": 8192, "gdn_decode": 32}[args.workload]
         obj.K = {"quantize": 5120, "gdn": 5120, "linear": 1024}.get(args.workload, 5120)
         obj.N = {"linear": 1024, "gdn": 12352}.get(args.workload, 0)
         obj.flops = 2.0 * obj.M * obj.N * obj.K
@@ -1115,7 +1263,9 @@ class _CpuOnly:
                      "gdn": f"gdn_inproj_m{obj.M}_n12352_k5120", "linear": f"linear_m{obj.M}_n1024_k1024",
                      "sweep": f"hybrid_sweep_496_linears_m{obj.M}",
                      "decode": f"decode_sweep_496_linears_m{obj.M}",
-                     "kv": f"kv_cache_fp8_m{obj.M}_w1024"}[args.workload]
+                     "kv": f"kv_cache_fp8_m{obj.M}_w1024",
+                     "gdn_rec": f"gdn_recurrence_t{obj.M}_seq{min(obj.M, 4096)}_hk16_hv32_d128",
+                     "gdn_decode": f"gdn_decode_b{obj.M}_hk16_hv32_d128"}[args.workload]
 
     def cpu_sample(self):
         return self.cls.cpu_sample(self.obj)

@@ -301,6 +301,41 @@ NVFP4_API nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf
                                             int64_t num_slots, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gdn_recurrence - the gated delta-rule recurrence of the Gated DeltaNet layers,
+ * fed by the gate epilogue of the fused in-projection (NVFP4_EPI_GDN_GATES):
+ *   for each sequence s, value head h and token t of the sequence, in order,
+ *     S <- exp(g[t,h]) * S + beta[t,h] * k_t (v_t - S^T k_t)^T
+ *     out[t, h*128 : h*128+128] = S^T q_t
+ *   with k_t, q_t the 128-vectors of key head h / (n_value_heads / n_key_heads) and v_t
+ *   that of value head h.  Source: blog section "Gated DeltaNetの仕組み" (the state
+ *   update, alpha = forget gate, beta = write strength); alpha = exp(g) follows the log-
+ *   space decay the gate epilogue produces (section 機構②).  The read-out S^T q with the
+ *   updated state is this library's reading (the pages give none); q and k are used as
+ *   given (no normalisation or scaling).  FP32 state and arithmetic.
+ *   q, k: device BF16 rows [tokens x ld_qk] (key head hk at column hk*128); v: device
+ *   BF16 [tokens x ld_v] (value head h at column h*128); q, k, v 16-byte aligned, ld_qk
+ *   and ld_v multiples of 8.  They may be column ranges of one projection output.
+ *   g, beta: device FP32 [tokens x ld_gate], head h at column h (the layout the gate
+ *   epilogue writes).  cu_seqlens: device int32 [n_seqs + 1], sequence s = tokens
+ *   cu_seqlens[s] .. cu_seqlens[s+1]-1 (empty sequences allowed); a sequence whose
+ *   bounds are not 0 <= start <= end <= tokens is skipped (state and out untouched) and
+ *   reported as NVFP4_ERR_DEVICE_INDEX by nvfp4_get_device_status.
+ *   state: device FP32 [n_seqs][n_value_heads][128][128], 16-byte aligned: entry
+ *   [s][h][j][i] holds S[i][j] (i over d_k, j over d_v).  Read as the initial state when
+ *   initial_state != 0 (else S starts at 0), overwritten with the final state.
+ *   out: device [tokens x ld_out] of out_kind NVFP4_OUT_BF16 (ld_out % 8 == 0) or
+ *   NVFP4_OUT_F32 (ld_out % 4 == 0), 16-byte aligned.  head_dim must be 128;
+ *   n_value_heads a multiple of n_key_heads; n_seqs, n_value_heads <= 65535.
+ *   Buffers must not overlap except q, k and v (read only).
+ */
+NVFP4_API nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int64_t ld_qk,
+                                              const void *v_bf16, int64_t ld_v, const float *g, const float *beta,
+                                              int64_t ld_gate, const int32_t *cu_seqlens, int64_t n_seqs,
+                                              int64_t tokens, int n_key_heads, int n_value_heads, int head_dim,
+                                              float *state, int initial_state, void *out, int64_t ld_out,
+                                              int out_kind, nvfp4_stream_t stream);
+
+/*
  * nvfp4_get_device_status - read and clear the device status word of the current
  * device.  Kernels never spin forever: every wait on an mbarrier has an iteration
  * limit, and a wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the

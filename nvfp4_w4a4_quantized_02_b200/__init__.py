@@ -15,7 +15,7 @@ from typing import Optional, Sequence
 __all__ = [
     "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
     "linear_splitk", "linear_splitk_noalloc", "splitk_default", "splitk_workspace_bytes",
-    "NOALLOC_SCRATCH_BYTES", "fold_segments", "fp8_scale", "kv_cache_fp8",
+    "NOALLOC_SCRATCH_BYTES", "fold_segments", "fp8_scale", "kv_cache_fp8", "gdn_recurrence",
     "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
 ]
 
@@ -55,7 +55,7 @@ _LIB = None
 SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
            "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
            "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_fold_segments",
-           "nvfp4_fp8_scale", "nvfp4_kv_cache_fp8", "nvfp4_get_device_status")
+           "nvfp4_fp8_scale", "nvfp4_kv_cache_fp8", "nvfp4_gdn_recurrence", "nvfp4_get_device_status")
 
 
 def lib():
@@ -103,6 +103,10 @@ def lib():
     L.nvfp4_kv_cache_fp8.restype = ctypes.c_int
     L.nvfp4_kv_cache_fp8.argtypes = [_c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
                                      _c_i64, _c_vp]
+    L.nvfp4_gdn_recurrence.restype = ctypes.c_int
+    L.nvfp4_gdn_recurrence.argtypes = [_c_vp, _c_vp, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_i64, _c_vp, _c_i64,
+                                       _c_i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_vp, ctypes.c_int,
+                                       _c_vp, _c_i64, ctypes.c_int, _c_vp]
     L.nvfp4_get_device_status.restype = ctypes.c_int
     L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     _LIB = L
@@ -340,6 +344,39 @@ def kv_cache_fp8(k, v, k_scale, v_scale, slots, k_cache, v_cache, stream=None):
                                     _c_vp(k_scale.data_ptr()), _c_vp(v_scale.data_ptr()), _c_vp(slots.data_ptr()),
                                     _c_vp(k_cache.data_ptr()), _c_vp(v_cache.data_ptr()), k_cache.shape[0],
                                     _stream(stream)), "nvfp4_kv_cache_fp8")
+
+
+def gdn_recurrence(q, k, v, g, beta, cu_seqlens, state, *, initial_state=True, out=None, out_dtype="bf16",
+                   stream=None):
+    """Gated delta-rule recurrence of the GDN layers over packed sequences.
+
+    q, k: BF16 [tokens, H_k * 128] (row-strided views allowed, e.g. column ranges of the
+    fused in-projection output); v: BF16 [tokens, H_v * 128]; g, beta: FP32 [tokens, H_v]
+    (row-strided, as the gate epilogue writes them); cu_seqlens: int32 [n_seqs + 1];
+    state: FP32 [n_seqs, H_v, 128, 128] with state[s, h, j, i] = S[i, j], read as the
+    initial state when ``initial_state`` and overwritten with the final one.  Returns
+    out [tokens, H_v * 128] (BF16 or FP32), out[t, h*128 + j] = (S_t^T q_t)_j."""
+    import torch
+    tokens = q.shape[0]
+    hk, hv = q.shape[1] // 128, v.shape[1] // 128
+    assert q.dtype == k.dtype == v.dtype == torch.bfloat16 and q.shape == k.shape and q.stride() == k.stride()
+    assert q.stride(1) == 1 and v.stride(1) == 1 and v.shape[0] == tokens
+    assert g.dtype == beta.dtype == torch.float32 and g.stride() == beta.stride() and g.shape[1] >= hv
+    assert cu_seqlens.dtype == torch.int32 and state.dtype == torch.float32 and state.is_contiguous()
+    n_seqs = cu_seqlens.shape[0] - 1
+    assert state.shape == (n_seqs, hv, 128, 128)
+    if out_dtype not in ("bf16", "f32"):
+        raise ValueError(f"out_dtype must be 'bf16' or 'f32', not {out_dtype!r}")
+    kind = OUT_KINDS[out_dtype]
+    if out is None:
+        out = torch.empty((tokens, hv * 128), device=q.device,
+                          dtype=torch.bfloat16 if out_dtype == "bf16" else torch.float32)
+    _check(lib().nvfp4_gdn_recurrence(_c_vp(q.data_ptr()), _c_vp(k.data_ptr()), q.stride(0), _c_vp(v.data_ptr()),
+                                      v.stride(0), _c_vp(g.data_ptr()), _c_vp(beta.data_ptr()), g.stride(0),
+                                      _c_vp(cu_seqlens.data_ptr()), n_seqs, tokens, hk, hv, 128,
+                                      _c_vp(state.data_ptr()), int(bool(initial_state)), _c_vp(out.data_ptr()),
+                                      out.stride(0), kind, _stream(stream)), "nvfp4_gdn_recurrence")
+    return out
 
 
 def device_status() -> int:

@@ -12,7 +12,6 @@
 namespace nvfp4 {
 
 constexpr int kKvThreads = 256;
-constexpr int kStatusBadIndex = 7;  // == NVFP4_ERR_DEVICE_INDEX
 
 struct KvArgs {
   const uint16_t *k, *v;  // BF16 [tokens x width], row stride ld elements

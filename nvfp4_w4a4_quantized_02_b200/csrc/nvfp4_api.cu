@@ -12,6 +12,7 @@
 #include "gemm.cuh"
 #include "fold.cuh"
 #include "kvcache.cuh"
+#include "gdn.cuh"
 
 using namespace nvfp4;
 
@@ -58,7 +59,11 @@ nvfp4_status_t current_device(DeviceInfo **info) {
         cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
             cudaSuccess ||
         cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes) !=
-            cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(gdn::recurrence_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(sizeof(gdn::Smem<32>))) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn::recurrence_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(sizeof(gdn::Smem<16>))) != cudaSuccess)
       return NVFP4_ERR_CUDA;
     {
       cudaLaunchConfig_t cfg = {};
@@ -579,6 +584,53 @@ nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_
   const int64_t cap = int64_t(dev->sms) * 16;
   const int grid = static_cast<int>(want < cap ? want : cap);
   kv_cache_fp8_kernel<<<grid, kKvThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
+nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int64_t ld_qk, const void *v_bf16,
+                                    int64_t ld_v, const float *g, const float *beta, int64_t ld_gate,
+                                    const int32_t *cu_seqlens, int64_t n_seqs, int64_t tokens, int n_key_heads,
+                                    int n_value_heads, int head_dim, float *state, int initial_state, void *out,
+                                    int64_t ld_out, int out_kind, nvfp4_stream_t stream) {
+  if (!q_bf16 || !k_bf16 || !v_bf16 || !g || !beta || !cu_seqlens || !state || !out) return NVFP4_ERR_INVALID_ARG;
+  if (n_seqs < 1 || tokens < 0 || n_key_heads < 1 || n_value_heads < 1 || n_value_heads % n_key_heads != 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (out_kind != NVFP4_OUT_BF16 && out_kind != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+  if (head_dim != gdn::kDim || n_seqs > 65535 || n_value_heads > 65535 || tokens > kMaxDim)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const int64_t wk = int64_t(n_key_heads) * gdn::kDim, wv = int64_t(n_value_heads) * gdn::kDim;
+  if (ld_qk < wk || ld_v < wv || ld_gate < n_value_heads || ld_out < wv) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(q_bf16, 16) || !aligned(k_bf16, 16) || !aligned(v_bf16, 16) || ld_qk % 8 != 0 || ld_v % 8 != 0 ||
+      !aligned(g, 4) || !aligned(beta, 4) || !aligned(cu_seqlens, 4) || !aligned(state, 16) || !aligned(out, 16) ||
+      ld_out % (out_kind == NVFP4_OUT_BF16 ? 8 : 4) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  gdn::Args a;
+  a.q = static_cast<const uint16_t *>(q_bf16);
+  a.k = static_cast<const uint16_t *>(k_bf16);
+  a.v = static_cast<const uint16_t *>(v_bf16);
+  a.ld_qk = ld_qk;
+  a.ld_v = ld_v;
+  a.g = g;
+  a.beta = beta;
+  a.ld_gate = ld_gate;
+  a.cu_seqlens = cu_seqlens;
+  a.tokens = tokens;
+  a.heads_per_key = n_value_heads / n_key_heads;
+  a.state = state;
+  a.initial = initial_state != 0;
+  a.out = out;
+  a.ld_out = ld_out;
+  a.out_fp32 = out_kind == NVFP4_OUT_F32;
+  const dim3 grid(gdn::kColBlocks, n_value_heads, static_cast<unsigned>(n_seqs));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // Short sequences (decode: about one token each) stage 16 tokens at a time, which
+  // keeps the shared-memory footprint, and so the occupancy, of the state-bound case.
+  if (tokens >= 16 * n_seqs)
+    gdn::recurrence_kernel<32><<<grid, gdn::kThreads, sizeof(gdn::Smem<32>), s>>>(a);
+  else
+    gdn::recurrence_kernel<16><<<grid, gdn::kThreads, sizeof(gdn::Smem<16>), s>>>(a);
   return launch_status();
 }
 

@@ -13,6 +13,7 @@ namespace nvfp4 {
 __device__ int g_device_status = 0;
 
 constexpr int kStatusTimeout = 5;          // == NVFP4_ERR_DEVICE_TIMEOUT
+constexpr int kStatusBadIndex = 7;         // == NVFP4_ERR_DEVICE_INDEX
 constexpr uint32_t kMaxWaitIters = 1u << 22;  // try_wait suspends between polls: >= ~0.1 s in total
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -20,7 +20,10 @@ Distributions follow the workloads the method is measured on:
   statistics the blog reports in its block-scaling mechanism section
   ("27BハイブリッドLLMを4ビットで動かす", section 機構①);
 * weights ~ N(0, 0.02), with per-segment multipliers where a fused module's
-  segments must carry global scales that differ (up to 16x).
+  segments must carry global scales that differ (up to 16x);
+* GDN recurrence inputs: unit-norm q / k heads, N(0,1) values, log-decays g <= 0 whose
+  per-head rates span the short to the very long memory horizons the blog's recurrence
+  section mentions (tens of thousands of tokens), write strengths beta in (0, 1).
 """
 from __future__ import annotations
 
@@ -28,7 +31,7 @@ import numpy as np
 
 __all__ = [
     "f32_to_bf16_bits", "bf16_to_f32", "outlier_activations", "student_t_activations",
-    "gaussian_weights", "segmented_weights", "gdn_gate_params",
+    "gaussian_weights", "segmented_weights", "gdn_gate_params", "gdn_recurrence_inputs",
     "GDN_INPROJ_SEGMENTS", "GDN_INPROJ_MULTIPLIERS",
 ]
 
@@ -117,3 +120,32 @@ def gdn_gate_params(n_heads: int = 32, seed: int = 7):
     a_log = rng.standard_normal(n_heads).astype(np.float32)
     dt_bias = rng.standard_normal(n_heads).astype(np.float32)
     return a_log, dt_bias
+
+
+def gdn_recurrence_inputs(seq_lens, n_key_heads: int = 16, n_value_heads: int = 32, seed: int = 11,
+                          ld: int | None = None, head_dim: int = 128):
+    """Packed sequences of GDN recurrence inputs laid out like the fused in-projection's
+    output rows: q at column 0, k at n_key_heads * head_dim, v after k; row width ``ld``
+    (default: just q | k | v).
+
+    q, k: each head an i.i.d. Gaussian vector scaled to unit length, then rounded to
+    BF16; v ~ N(0, 1) in BF16; g[t, h] = -c_h * U(0.5, 1.5) with per-head rates c_h
+    log-uniform in [2e-5, 0.5] (float32); beta ~ U(0.05, 1) (float32).
+    Returns dict(rows=uint16 [T, ld], q_col, k_col, v_col, g, beta, cu_seqlens=int32)."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(seq_lens, np.int64)
+    T = int(lens.sum())
+    wk, wv = n_key_heads * head_dim, n_value_heads * head_dim
+    ld = 2 * wk + wv if ld is None else ld
+    assert ld >= 2 * wk + wv
+    rows = np.zeros((T, ld), np.uint16)
+    for col in (0, wk):
+        x = rng.standard_normal((T, n_key_heads, head_dim))
+        x /= np.linalg.norm(x, axis=-1, keepdims=True)
+        rows[:, col:col + wk] = f32_to_bf16_bits(x.reshape(T, wk).astype(np.float32))
+    rows[:, 2 * wk:2 * wk + wv] = f32_to_bf16_bits(rng.standard_normal((T, wv)).astype(np.float32))
+    rate = np.exp(rng.uniform(np.log(2e-5), np.log(0.5), n_value_heads))
+    g = (-rate[None, :] * rng.uniform(0.5, 1.5, (T, n_value_heads))).astype(np.float32)
+    beta = rng.uniform(0.05, 1.0, (T, n_value_heads)).astype(np.float32)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return dict(rows=rows, q_col=0, k_col=wk, v_col=2 * wk, g=g, beta=beta, cu_seqlens=cu)

@@ -92,3 +92,27 @@ def test_splitk_helpers_without_device(L):
     # invalid sizes are rejected before any device query
     assert L.nvfp4_splitk_default(0, 256, 512) == 0
     assert L.nvfp4_splitk_default(8, 256, 300) == 0
+
+
+def test_gdn_recurrence_rejects_bad_arguments_without_launch(L):
+    vp = ctypes.c_void_p
+    f = vp(1 << 20)  # never dereferenced: validation fails first
+
+    def call(q=f, ld_qk=256, ld_v=512, ld_gate=4, n_seqs=1, tokens=8, hk=2, hv=4, d=128, state=f, out=f,
+             ld_out=512, kind=0):
+        return L.nvfp4_gdn_recurrence(q, f, ld_qk, f, ld_v, f, f, ld_gate, f, n_seqs, tokens, hk, hv, d, state, 1,
+                                      out, ld_out, kind, None)
+    assert call(q=None) == 1
+    assert call(d=64) == 2                        # head_dim must be 128
+    assert call(hk=3, hv=4) == 1                  # value heads not a multiple of key heads
+    assert call(n_seqs=0) == 1
+    assert call(n_seqs=70000) == 2
+    assert call(kind=2) == 1                      # NVFP4 output not offered
+    assert call(ld_qk=128) == 1                   # 2 key heads need 256 columns
+    assert call(ld_v=256) == 1
+    assert call(ld_gate=3) == 1
+    assert call(ld_out=500) == 1
+    assert call(q=vp((1 << 20) + 8)) == 3         # q not 16-byte aligned
+    assert call(ld_qk=260) == 3                   # row stride not a multiple of 8 BF16
+    assert call(state=vp((1 << 20) + 4)) == 3
+    assert call(ld_out=516) == 3                  # BF16 out rows must stay 16-byte aligned
