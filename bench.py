@@ -152,7 +152,8 @@ def sources_hash(files):
 
 def load_traffic(key):
     """DRAM bytes per launch of ``key`` (``kernel@workload``) from the committed ncu
-    summary ``profiles/traffic.json``, or None when the kernel's sources changed since."""
+    summary ``profiles/traffic.json``, or None when the kernel's sources (the device
+    code files listed with the entry) changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             ent = json.load(f).get(key)
@@ -389,7 +390,7 @@ class MLPBlock(Workload):
         self.l2_note = (f"inputs larger than L2 (X {M * H * 2 / 1e6:.0f} MB, H {M * I * 0.5625 / 1e6:.0f} MB, "
                         f"out {M * H * 2 / 1e6:.0f} MB per step)")
         self.dominant = ("gemm_gate_up", self.f_gu, "tensor",
-                         "gemm_kernel (gate|up, SiLU*mul, NVFP4 requant epilogue)")
+                         "gemm2_kernel (CTA pair; gate|up, SiLU*mul, NVFP4 requant epilogue)")
         self.phases = {"global_scale": ("GB/s", 2.0 * M * H), "quantize": ("GB/s", 2.5625 * M * H),
                        "gemm_gate_up": ("TFLOP/s", self.f_gu), "gemm_down": ("TFLOP/s", self.f_d)}
 
@@ -501,7 +502,7 @@ class GDNInProj(Workload):
         self.launches_per_step = 4
         self.l2_note = (f"per-step working set {(M * K * 2.5625 + self.N * K * 0.5625 + M * self.N * 2) / 1e6:.0f} MB "
                         "> L2 (X, its codes, W, BF16 out)")
-        self.dominant = ("gemm", self.flops, "tensor", "gemm_kernel (6 segments, GDN gate epilogue)")
+        self.dominant = ("gemm", self.flops, "tensor", "gemm2_kernel (CTA pair; 6 segments, GDN gate epilogue)")
         self.phases = {"global_scale": ("GB/s", 2.0 * M * K), "quantize": ("GB/s", 2.5625 * M * K),
                        "gemm": ("TFLOP/s", self.flops)}
         torch.cuda.synchronize()
@@ -684,7 +685,7 @@ class HybridSweep(Workload):
                                 for t in ([v[0]] if isinstance(v, tuple) else [v]))
         self.l2_note = f"weights {self.packed_bytes / 2**30:.2f} GiB packed, streamed once per step (> L2)"
         self.dominant = ("gemm_gate_up", self.f_gu, "tensor",
-                         "gemm_kernel (MLP gate|up, SiLU*mul, NVFP4 requant epilogue)")
+                         "gemm2_kernel (CTA pair; MLP gate|up, SiLU*mul, NVFP4 requant epilogue)")
         self.phases = {"quantize": ("GB/s", 2.5625 * M * (128 * H + 48 * 4096 + 16 * 6144)),
                        "gemm_gdn_in": ("TFLOP/s", 48 * 2.0 * M * 12352 * H),
                        "gemm_gdn_out": ("TFLOP/s", 48 * 2.0 * M * H * 4096),
@@ -925,7 +926,7 @@ class GDNDecode(GDNRecurrence):
         self.state.copy_(0.3 * torch.randn(self.state.shape, generator=g, device="cuda"))
         self.bytes = M * (32 * 2 * 128 * 128 * 4 + 8192 * 2 + 2 * 32 * 4 + 4096 * 2) + 4.0 * (M + 1)
         self.l2_note = f"states {self.state.numel() * 4 / 1e6:.0f} MB read and written per step (> L2)"
-        self.dominant = ("gdn_recurrence", self.bytes, "hbm", "gdn recurrence_kernel<8> (state read + write)")
+        self.dominant = ("gdn_recurrence", self.bytes, "hbm", "gdn recurrence_kernel<16> (state read + write)")
         self.phases = {"gdn_recurrence": ("GB/s", self.bytes)}
 
     def work(self):
