@@ -6,6 +6,8 @@ checked on sampled output rows that the oracle computes one by one.
   own global scale (multipliers 1|2|4|8|16|1), gate epilogue.
 * MLP block: X [32768 x 5120] (Student-t(3), 8 hot channels x100), gate|up
   [2 x 17408 x 5120] with SiLU*mul and NVFP4 re-quantisation, down [5120 x 17408].
+* The other linears of the 496-linear sweep at M = 4096: GDN output projection,
+  fused attention q|k|v (three modules, three global scales), attention output.
 """
 import numpy as np
 import pytest
@@ -143,4 +145,64 @@ def test_mlp_block_full_size_sampled_rows(nv):
     out = nv.linear(h_op, w_d, out_dtype="bf16")
     torch.cuda.synchronize()
     assert_gemm_close(out[rows_t], out_ref)
+    assert nv.device_status() == 0
+
+
+# The remaining linear shapes of the 496-linear sweep, at its M = 4096 prefill size
+# (the CTA-pair kernel, as the sweep launches them): the GDN output projection
+# (4096 -> 5120), the attention q|k|v projection fused as one GEMM of three modules
+# with their own global scales (5120 -> 6144 | 1024 | 1024), and the attention output
+# projection (6144 -> 5120).  Inputs: Student-t(3) activations standing in for the
+# layer input / mixer output, N(0, 0.02) weights (k and v modules x2 and x4 so that
+# the three global scales differ).
+SWEEP_SHAPES = [
+    ("gdn_out", 4096, [("o", 5120, 1.0)]),
+    ("attn_qkv", 5120, [("q", 6144, 1.0), ("k", 1024, 2.0), ("v", 1024, 4.0)]),
+    ("attn_o", 6144, [("o", 5120, 1.0)]),
+]
+
+
+def _sample_cols(n, n_random, seed):
+    """Tile-boundary weight rows (output columns) of a module plus seeded random ones."""
+    fixed = [0, 1, 127, 128, 255, 256, n // 2, n - 257, n - 256, n - 129, n - 128, n - 1]
+    rng = np.random.default_rng(seed)
+    cols = np.unique(np.concatenate([fixed, rng.choice(n, n_random, replace=False)]))
+    return cols[(cols >= 0) & (cols < n)]
+
+
+@pytest.mark.parametrize("name,K,mods", SWEEP_SHAPES, ids=[s[0] for s in SWEEP_SHAPES])
+def test_sweep_linear_shapes_sampled_rows(nv, name, K, mods):
+    """Sampled rows x sampled output columns of each module (every module's global
+    scale taken over its whole weight), against the oracle."""
+    import torch
+    M = 4096
+    xb = synth.student_t_activations(M, K, seed=20)
+    wbs = [synth.gaussian_weights(n, K, seed=21 + i, std=0.02 * m) for i, (_, n, m) in enumerate(mods)]
+    rows = _sample_rows(M, 24, seed=5)
+
+    gsa = oracle.global_scale(synth.bf16_to_f32(xb))
+    ca, sa = _oracle_rows(xb, rows, gsa)
+    oc, os_, oseg, cols, n0, off = [], [], [], [], 0, 0
+    for i, wb in enumerate(wbs):
+        gw = oracle.global_scale(synth.bf16_to_f32(wb))
+        cm = _sample_cols(wb.shape[0], 40, seed=30 + i)
+        c, s_ = oracle.quantize(synth.bf16_to_f32(wb[cm]), np.float32(gw))
+        oc.append(c), os_.append(s_), oseg.append((n0, n0 + len(cm), np.float32(gw)))
+        cols.append(off + cm)
+        n0 += len(cm)
+        off += wb.shape[0]
+    y = oracle.linear(ca, sa, gsa, np.concatenate(oc), np.concatenate(os_), oseg)
+    cols = np.concatenate(cols)
+
+    a = nv.quantize(to_dev_bf16(xb))
+    if len(wbs) == 1:
+        w = nv.quantize(to_dev_bf16(wbs[0]))
+        out = nv.linear(a, w, out_dtype="bf16")
+    else:
+        w, dsegs = nv.quantize_fused([to_dev_bf16(wb) for wb in wbs])
+        out = nv.linear(a, w, segments=dsegs, out_dtype="bf16")
+    torch.cuda.synchronize()
+    assert float(a.gs.item()) == float(gsa)
+    got = out[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()]
+    assert_gemm_close(got, y)
     assert nv.device_status() == 0
