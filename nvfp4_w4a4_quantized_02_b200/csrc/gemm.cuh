@@ -185,9 +185,13 @@ __device__ __forceinline__ float seg_alpha(const Ctrl<STAGES> &c, int nseg, int 
   return a;
 }
 
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+// Gate and activation functions with the hardware approximations (relative error of
+// order 1e-6: far below the BF16 store and the 1e-3 bar of the gates).  softplus uses
+// the stable form max(x, 0) + log(1 + e^-|x|); 1 + e^-|x| lies in (1, 2], where the
+// logarithm's absolute error stays below 1e-6.
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float silu_mul_f(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
-__device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x))); }
+__device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))); }
 
 // Store 16 consecutive output values of one row.
 __device__ __forceinline__ void store16(const Params &p, int row, int col, const float (&y)[16]) {
@@ -236,21 +240,21 @@ __device__ __forceinline__ void store64_nvfp4(const Params &p, const float *inv_
   *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, col / 64, p.out_kb_atoms)) = sfword;
 }
 
-// GDN gates of the 64 outputs starting at column cg of one row, for the columns that
-// fall in the beta or alpha head blocks.  Kept out of line: only the N-tile holding
-// the head blocks gets here, and the unrolled epilogue stays small.
-__device__ __noinline__ void gdn_gates64(const Params &p, int row, int cg, float *y) {
+// GDN gates of the 64 outputs starting at column cg of one row, in place in the
+// caller's registers, for the columns that fall in the beta or alpha head blocks
+// (blocks are disjoint; only the N-tile holding them gets here).  Unrolled over the
+// 64 columns so that the exp / log / division chains of neighbouring columns overlap.
+__device__ __forceinline__ void gdn_gates64(const Params &p, int row, int cg, float (&y)[64]) {
+#pragma unroll
   for (int i = 0; i < 64; ++i) {
     const int n = cg + i;
     if (n >= p.beta_begin && n < p.beta_begin + p.n_heads) {
-      const float bt = sigmoid_f(y[i]);
-      y[i] = bt;
-      if (p.beta_out) p.beta_out[(int64_t)row * p.n_heads + (n - p.beta_begin)] = bt;
+      y[i] = sigmoid_f(y[i]);
+      if (p.beta_out) p.beta_out[(int64_t)row * p.n_heads + (n - p.beta_begin)] = y[i];
     } else if (n >= p.alpha_begin && n < p.alpha_begin + p.n_heads) {
       const int hh = n - p.alpha_begin;
-      const float g = -expf(__ldg(p.A_log + hh)) * softplus_f(y[i] + __ldg(p.dt_bias + hh));
-      y[i] = g;
-      if (p.g_out) p.g_out[(int64_t)row * p.n_heads + hh] = g;
+      y[i] = -__expf(__ldg(p.A_log + hh)) * softplus_f(y[i] + __ldg(p.dt_bias + hh));
+      if (p.g_out) p.g_out[(int64_t)row * p.n_heads + hh] = y[i];
     }
   }
 }
@@ -330,14 +334,8 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
       for (int i = 0; i < 16; ++i) y[16 * b + i] = a * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
     }
     if (p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + 64 > p.beta_begin) ||
-                               (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin))) {
-      float t[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) t[i] = y[i];
-      gdn_gates64(p, row, cg, t);
-#pragma unroll
-      for (int i = 0; i < 64; ++i) y[i] = t[i];
-    }
+                               (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin)))
+      gdn_gates64(p, row, cg, y);
     if (p.out_kind == OUT_NVFP4) {
       store64_nvfp4(p, c.inv_out, row, cg, y, gs_out);
     } else {
@@ -769,7 +767,7 @@ __device__ __forceinline__ void partial_sum16(const Params &p, int row, int col,
   }
 }
 
-__global__ void __launch_bounds__(REDUCE_THREADS) splitk_epilogue_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(REDUCE_THREADS, 1) splitk_epilogue_kernel(const __grid_constant__ Params p) {
   __shared__ Ctrl<1> c;  // segment alphas and the NVFP4 output table
   load_segments(p, c);
   __syncthreads();
@@ -809,14 +807,8 @@ __global__ void __launch_bounds__(REDUCE_THREADS) splitk_epilogue_kernel(const _
     for (int i = 0; i < 16; ++i) y[16 * b + i] = t[i];
   }
   if (p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + 64 > p.beta_begin) ||
-                             (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin))) {
-    float t[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) t[i] = y[i];
-    gdn_gates64(p, row, cg, t);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) y[i] = t[i];
-  }
+                             (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin)))
+    gdn_gates64(p, row, cg, y);
   if (p.out_kind == OUT_NVFP4) {
     store64_nvfp4(p, c.inv_out, row, cg, y, __ldg(p.gs_out));
   } else {
