@@ -215,9 +215,9 @@ NVFP4_API nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const flo
 NVFP4_API size_t nvfp4_splitk_workspace_bytes(int64_t M, int64_t N, int split_k);
 
 /* The split count the library would choose for an M x N x K linear on the current
- * device (>= 1, <= K/256): 1 unless the output tiles fill under a quarter of the SMs
- * and K has at least 32 tiles of 256; then enough units to fill the SMs once, with at
- * least 8 K tiles per split.  0 for invalid sizes or when the device cannot be
+ * device (>= 1, <= K/256): as many splits as keep all (output tile of 128 x 256, K
+ * range) work units in one wave on the SMs, i.e. SMs / tiles rounded down, with at
+ * least 4 K tiles of 256 per split.  0 for invalid sizes or when the device cannot be
  * queried. */
 NVFP4_API int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K);
 

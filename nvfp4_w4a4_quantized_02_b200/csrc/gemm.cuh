@@ -240,13 +240,14 @@ __device__ __forceinline__ void store64_nvfp4(const Params &p, const float *inv_
   *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, col / 64, p.out_kb_atoms)) = sfword;
 }
 
-// GDN gates of the 64 outputs starting at column cg of one row, in place in the
+// GDN gates of the W outputs starting at column cg of one row, in place in the
 // caller's registers, for the columns that fall in the beta or alpha head blocks
 // (blocks are disjoint; only the N-tile holding them gets here).  Unrolled over the
-// 64 columns so that the exp / log / division chains of neighbouring columns overlap.
-__device__ __forceinline__ void gdn_gates64(const Params &p, int row, int cg, float (&y)[64]) {
+// columns so that the exp / log / division chains of neighbouring columns overlap.
+template <int W>
+__device__ __forceinline__ void gdn_gates(const Params &p, int row, int cg, float (&y)[W]) {
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
+  for (int i = 0; i < W; ++i) {
     const int n = cg + i;
     if (n >= p.beta_begin && n < p.beta_begin + p.n_heads) {
       y[i] = sigmoid_f(y[i]);
@@ -257,6 +258,12 @@ __device__ __forceinline__ void gdn_gates64(const Params &p, int row, int cg, fl
       if (p.g_out) p.g_out[(int64_t)row * p.n_heads + hh] = y[i];
     }
   }
+}
+
+// Whether columns [cg, cg + w) touch a GDN head block.
+__device__ __forceinline__ bool touches_gates(const Params &p, int cg, int w) {
+  return p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + w > p.beta_begin) ||
+                                (cg < p.alpha_begin + p.n_heads && cg + w > p.alpha_begin));
 }
 
 // TMEM -> registers for one epilogue warp: 32 lanes of quadrant q, 128 columns
@@ -333,9 +340,7 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
 #pragma unroll
       for (int i = 0; i < 16; ++i) y[16 * b + i] = a * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
     }
-    if (p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + 64 > p.beta_begin) ||
-                               (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin)))
-      gdn_gates64(p, row, cg, y);
+    if (touches_gates(p, cg, 64)) gdn_gates<64>(p, row, cg, y);
     if (p.out_kind == OUT_NVFP4) {
       store64_nvfp4(p, c.inv_out, row, cg, y, gs_out);
     } else {
@@ -746,81 +751,95 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ======================================================= split-K epilogue
 // Sums the splits' partials and applies the epilogue of the linear: one thread per
-// 64 output columns of one row (one scale word of an NVFP4 output).  Rows past M up
-// to the next multiple of 128 only write zero scale words (NVFP4 output).
+// 16 output columns of one row (one E4M3 block of an NVFP4 output), so that a
+// decode-size output (tens of rows) still spreads over thousands of threads; rows
+// past M up to the next multiple of 128 only write zero scale bytes (NVFP4 output).
 constexpr int REDUCE_THREADS = 256;
 
-// 16 consecutive column sums (col % 16 == 0, col + 16 <= N).
+// 16 consecutive column sums (col % 16 == 0, col + 16 <= N), added split by split in
+// order, with two splits' loads in flight.
 __device__ __forceinline__ void partial_sum16(const Params &p, int row, int col, float (&y)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) y[i] = 0.0f;
-  for (int sp = 0; sp < p.splits; ++sp) {
-    const float4 *src = reinterpret_cast<const float4 *>(p.partial + ((int64_t)sp * p.M + row) * p.N + col);
+  const int64_t stride = (int64_t)p.M * p.N;
+  const float4 *src = reinterpret_cast<const float4 *>(p.partial + (int64_t)row * p.N + col);
+  int sp = 0;
+  for (; sp + 2 <= p.splits; sp += 2) {
+    const float4 *s0 = src + sp * (stride / 4), *s1 = src + (sp + 1) * (stride / 4);
+    float4 a[4], b[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 v = src[i];
-      y[4 * i] += v.x;
-      y[4 * i + 1] += v.y;
-      y[4 * i + 2] += v.z;
-      y[4 * i + 3] += v.w;
+      a[i] = s0[i];
+      b[i] = s1[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      y[4 * i] += a[i].x, y[4 * i + 1] += a[i].y, y[4 * i + 2] += a[i].z, y[4 * i + 3] += a[i].w;
+      y[4 * i] += b[i].x, y[4 * i + 1] += b[i].y, y[4 * i + 2] += b[i].z, y[4 * i + 3] += b[i].w;
     }
   }
+  if (sp < p.splits) {
+    const float4 *s0 = src + sp * (stride / 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 a = s0[i];
+      y[4 * i] += a.x, y[4 * i + 1] += a.y, y[4 * i + 2] += a.z, y[4 * i + 3] += a.w;
+    }
+  }
+}
+
+// Re-quantise 16 consecutive outputs (one block) of one row: the per-block arithmetic
+// of store64_nvfp4.
+__device__ __forceinline__ void store16_nvfp4(const Params &p, const float *inv_out, int row, int col,
+                                              const float (&y)[16], float gs_out) {
+  float x[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    x[i] = __bfloat162float(__float2bfloat16_rn(y[i]));
+    amax = fmaxf(amax, fabsf(x[i]));
+  }
+  const uint32_t sf = block_scale_byte(amax, gs_out);
+  const float inv = inv_out[sf & 127];
+  *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.out) + (int64_t)row * (p.Nout / 2) + col / 2) =
+      make_uint2(encode8(x, inv), encode8(x + 8, inv));
+  p.out_scales[scale_word_offset(row, col / 64, p.out_kb_atoms) + (col / 16) % 4] = static_cast<uint8_t>(sf);
 }
 
 __global__ void __launch_bounds__(REDUCE_THREADS, 1) splitk_epilogue_kernel(const __grid_constant__ Params p) {
   __shared__ Ctrl<1> c;  // segment alphas and the NVFP4 output table
   load_segments(p, c);
   __syncthreads();
-  const int groups = (p.Nout + 63) / 64;
+  const int blocks = p.Nout / 16;  // Nout % 16 == 0
   const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (int64_t)(p.M + 127) / 128 * 128 : p.M;
   const int64_t idx = (int64_t)blockIdx.x * REDUCE_THREADS + threadIdx.x;
-  if (idx >= rows_cover * groups) return;
-  const int row = static_cast<int>(idx / groups);
-  const int cg = static_cast<int>(idx - (int64_t)row * groups) * 64;
+  if (idx >= rows_cover * blocks) return;
+  const int row = static_cast<int>(idx / blocks);
+  const int col = static_cast<int>(idx - (int64_t)row * blocks) * 16;
   if (row >= p.M) {
-    *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, cg / 64, p.out_kb_atoms)) = 0u;
+    p.out_scales[scale_word_offset(row, col / 64, p.out_kb_atoms) + (col / 16) % 4] = 0;
     return;
   }
-  float y[64];
+  float y[16];
+  if (p.mode == MODE_SILU_MUL) {
+    float u[16];
+    partial_sum16(p, row, col, y);
+    partial_sum16(p, row, p.up_row0 + col, u);
+    const float ag = seg_alpha(c, p.nseg, col);
+    const float au = seg_alpha(c, p.nseg, p.up_row0 + col);
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const int col = cg + 16 * b;
-    float t[16];
-    if (col >= p.Nout) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) t[i] = 0.0f;
-    } else if (p.mode == MODE_SILU_MUL) {
-      float u[16];
-      partial_sum16(p, row, col, t);
-      partial_sum16(p, row, p.up_row0 + col, u);
-      const float ag = seg_alpha(c, p.nseg, col);
-      const float au = seg_alpha(c, p.nseg, p.up_row0 + col);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) t[i] = silu_mul_f(ag * t[i], au * u[i]);
-    } else {
-      partial_sum16(p, row, col, t);
-      const float a = seg_alpha(c, p.nseg, col);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) t[i] *= a;
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) y[16 * b + i] = t[i];
-  }
-  if (p.mode == MODE_GDN && ((cg < p.beta_begin + p.n_heads && cg + 64 > p.beta_begin) ||
-                             (cg < p.alpha_begin + p.n_heads && cg + 64 > p.alpha_begin)))
-    gdn_gates64(p, row, cg, y);
-  if (p.out_kind == OUT_NVFP4) {
-    store64_nvfp4(p, c.inv_out, row, cg, y, __ldg(p.gs_out));
+    for (int i = 0; i < 16; ++i) y[i] = silu_mul_f(ag * y[i], au * u[i]);
   } else {
+    partial_sum16(p, row, col, y);
+    const float a = seg_alpha(c, p.nseg, col);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      if (cg + 16 * b < p.Nout) {
-        float yy[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) yy[i] = y[16 * b + i];
-        store16(p, row, cg + 16 * b, yy);
-      }
-    }
+    for (int i = 0; i < 16; ++i) y[i] *= a;
+  }
+  if (touches_gates(p, col, 16)) gdn_gates<16>(p, row, col, y);
+  if (p.out_kind == OUT_NVFP4) {
+    store16_nvfp4(p, c.inv_out, row, col, y, __ldg(p.gs_out));
+  } else {
+    store16(p, row, col, y);
   }
 }
 

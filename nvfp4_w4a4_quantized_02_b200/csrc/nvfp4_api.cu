@@ -256,18 +256,17 @@ nvfp4_status_t prepare_linear(const nvfp4_operand_t *A, const float *gs_a, const
   return NVFP4_OK;
 }
 
-// Split count of the split-K linear.  Splitting pays only when few output tiles would
-// leave most SMs idle for a long K loop: the partial sums and the second kernel cost
-// about as much as a short GEMM (measured at 32 rows: the 5120 x 17408 projection gains
-// with 7 splits; 12352 x 5120, 5120 x 4096 and 5120 x 6144 lose).  So: more than one
-// split only when the tiles fill under a quarter of the SMs and K has >= 32 tiles; then
-// as many splits as fill the SMs once, keeping >= 8 K tiles per split.
+// Split count of the split-K linear: as many splits as keep all work units in one
+// wave on the SMs (SMs / tiles, rounded down), with at least 4 K tiles (1024 K) per
+// split.  Measured on the 496-linear decode step at 32 rows (one CUDA graph per step):
+// about 6 ms with a one-wave fill against 7.3-7.5 ms when only the 17408-long down
+// projection was split; a second wave (the MLP gate|up, 136 tiles, split twice) cost
+// 29 instead of 24 us per launch, and 2 K tiles per split was slower again.
 int default_splits(int64_t M, int64_t N, int64_t K, int sms) {
   const int64_t tiles = (M + gemm::BM - 1) / gemm::BM * ((N + gemm::BN - 1) / gemm::BN);
   const int64_t k_tiles = K / gemm::BK;
-  if (tiles * 4 >= sms || k_tiles < 32) return 1;
   int64_t s = sms / tiles;
-  if (s > k_tiles / 8) s = k_tiles / 8;
+  if (s > k_tiles / 4) s = k_tiles / 4;
   return static_cast<int>(s < 1 ? 1 : s);
 }
 
@@ -290,7 +289,7 @@ nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvf
   gemm_kernel<<<grid, NUM_THREADS, Plan1::BYTES, st>>>(tmA, tmB, p);
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (p.M + 127) / 128 * 128 : p.M;
-  const int64_t threads = rows_cover * ((p.Nout + 63) / 64);
+  const int64_t threads = rows_cover * (p.Nout / 16);  // one thread per 16-column block
   const int64_t blocks = (threads + REDUCE_THREADS - 1) / REDUCE_THREADS;
   if (blocks > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   splitk_epilogue_kernel<<<static_cast<unsigned>(blocks), REDUCE_THREADS, 0, st>>>(p);

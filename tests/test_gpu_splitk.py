@@ -28,6 +28,7 @@ def _sync():
 def test_down_proj_decode_full_size(nv):
     """32 decode tokens through the MLP down projection (5120 x 17408): FP32 and BF16
     outputs against the oracle, with the library's split count and with splits 1 and 5."""
+    import torch
     M, N, K = 32, 5120, 17408
     xb = synth.student_t_activations(M, K, seed=40)
     wb = synth.gaussian_weights(N, K, seed=41)
@@ -38,8 +39,15 @@ def test_down_proj_decode_full_size(nv):
     w = nv.quantize(to_dev_bf16(wb))
     s_def = nv.splitk_default(M, N, K)
     assert 1 < s_def <= K // 256  # 20 output tiles, 68 K tiles: the split pays here
-    assert nv.splitk_default(M, 34816, 5120) == 1  # 136 tiles already fill the SMs
-    assert nv.splitk_default(M, 5120, 4096) == 1  # 16 K tiles: too short to split
+    # the rule: SMs // tiles splits (one wave of work units), with >= 4 K tiles per split
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+
+    def rule(m, n, k):
+        tiles = -(-m // 128) * -(-n // 256)
+        return max(1, min(k // 256 // 4, sms // tiles))
+    for shape in [(M, N, K), (M, 34816, 5120), (M, 5120, 4096), (M, 12352, 5120), (4096, 5120, 4096),
+                  (M, 1024, 512)]:
+        assert nv.splitk_default(*shape) == rule(*shape), shape
     for s in (s_def, 1, 5):
         y32 = nv.linear_splitk(a, w, out_dtype="f32", split_k=s)
         y16 = nv.linear_splitk(a, w, out_dtype="bf16", split_k=s)
