@@ -27,6 +27,8 @@ struct FoldArgs {
 __global__ void __launch_bounds__(kFoldThreads) fold_scales_kernel(const __grid_constant__ FoldArgs a) {
   __shared__ float ratio[16];
   __shared__ float gs_c;
+  grid_dep_wait();
+  grid_dep_launch();
   if (threadIdx.x == 0) {
     float m = __ldg(a.gs[0]);
     for (int i = 1; i < a.nseg; ++i) m = fminf(m, __ldg(a.gs[i]));

@@ -210,6 +210,8 @@ __global__ void __launch_bounds__(kThreads) recurrence_kernel(const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int jl = 2 * (warp * (32 / kLanes) + lane / kLanes);  // first of the thread's two columns
   const int r = lane % kLanes;                                // row group: rows 16 r .. 16 r + 15
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t start = __ldg(a.cu_seqlens + b), end = __ldg(a.cu_seqlens + b + 1);
   if (start < 0 || end < start || end > a.tokens) {
     if (threadIdx.x == 0) atomicCAS(&g_device_status, 0, kStatusBadIndex);

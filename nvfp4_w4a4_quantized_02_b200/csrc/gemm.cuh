@@ -481,11 +481,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
   }
-  load_segments(p, c);
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  grid_dep_wait();  // operands, scales and global scales may come from the previous kernel
+  grid_dep_launch();
+  load_segments(p, c);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -640,11 +642,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tensormap(&tmSFA);
     prefetch_tensormap(&tmSFB);
   }
-  load_segments(p, c);
   if (warp == 1) {
     tmem_alloc_cg2(&c.tmem_base, TMEM_COLS);
     tmem_relinquish_cg2();
   }
+  grid_dep_wait();  // operands, scales and global scales may come from the previous kernel
+  grid_dep_launch();
+  load_segments(p, c);
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before either signals the other
@@ -808,6 +812,8 @@ __device__ __forceinline__ void store16_nvfp4(const Params &p, const float *inv_
 
 __global__ void __launch_bounds__(REDUCE_THREADS, 1) splitk_epilogue_kernel(const __grid_constant__ Params p) {
   __shared__ Ctrl<1> c;  // segment alphas and the NVFP4 output table
+  grid_dep_wait();  // the partial sums come from the previous kernel
+  grid_dep_launch();
   load_segments(p, c);
   __syncthreads();
   const int blocks = p.Nout / 16;  // Nout % 16 == 0

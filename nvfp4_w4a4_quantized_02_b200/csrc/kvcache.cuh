@@ -38,6 +38,8 @@ __device__ __forceinline__ uint4 fp8_chunk(const uint4 &w0, const uint4 &w1, flo
 }
 
 __global__ void __launch_bounds__(kKvThreads) kv_cache_fp8_kernel(const __grid_constant__ KvArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   const float k_inv = __frcp_rn(__ldg(a.k_scale)), v_inv = __frcp_rn(__ldg(a.v_scale));
   const int64_t per_row = a.width / 16;  // 16-element chunks per row
   // chunk idx = token * per_row + column chunk: shifts when per_row is a power of two
@@ -67,6 +69,8 @@ __global__ void __launch_bounds__(kKvThreads) kv_cache_fp8_kernel(const __grid_c
 
 // scale = fl32(amax / 448); amax == 0 -> 1.  In place: amax bits in, scale out.
 __global__ void fp8_scale_finalize_kernel(float *scale) {
+  grid_dep_wait();
+  grid_dep_launch();
   const float amax = *scale;
   *scale = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
 }

@@ -158,6 +158,36 @@ inline nvfp4_status_t launch_status() {
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Launches `kernel` with programmatic stream serialization: it may begin (shared
+// memory, barriers, TMEM) while the previous kernel on the stream finishes, and waits
+// for it in griddepcontrol.wait before touching global memory (every kernel of the
+// library does).  In a CUDA graph of many small launches (a decode step) this hides
+// most of each launch's latency and prologue.  cluster_x > 1 adds a cluster shape.
+template <typename... KArgs, typename... Args>
+nvfp4_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          unsigned cluster_x, Args &&...args) {
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
 // Validates the arguments of a linear and fills everything of Params but the tiling.
@@ -286,14 +316,13 @@ nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvf
   const int64_t units = int64_t(p.m_tiles) * p.n_tiles * p.splits;
   if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
-  gemm_kernel<<<grid, NUM_THREADS, Plan1::BYTES, st>>>(tmA, tmB, p);
-  if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (nvfp4_status_t e = launch_pdl(gemm_kernel, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p))
+    return e;
   const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (p.M + 127) / 128 * 128 : p.M;
   const int64_t threads = rows_cover * (p.Nout / 16);  // one thread per 16-column block
   const int64_t blocks = (threads + REDUCE_THREADS - 1) / REDUCE_THREADS;
   if (blocks > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  splitk_epilogue_kernel<<<static_cast<unsigned>(blocks), REDUCE_THREADS, 0, st>>>(p);
-  return launch_status();
+  return launch_pdl(splitk_epilogue_kernel, dim3(static_cast<unsigned>(blocks)), dim3(REDUCE_THREADS), 0, st, 1, p);
 }
 
 // ------------------------------------------------- scratch for callers that cannot allocate
@@ -365,9 +394,8 @@ nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols
   const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
   const int64_t cap = int64_t(dev->sms) * 8;
   const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
-  amax_kernel<<<grid, kAmaxThreads, 0, s>>>(a);
-  global_scale_finalize_kernel<<<1, 1, 0, s>>>(gs_out);
-  return launch_status();
+  if (nvfp4_status_t e = launch_pdl(amax_kernel, dim3(grid), dim3(kAmaxThreads), 0, s, 1, a)) return e;
+  return launch_pdl(global_scale_finalize_kernel, dim3(1), dim3(1), 0, s, 1, gs_out);
 }
 
 nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, const float *gs,
@@ -397,8 +425,8 @@ nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t col
   a.n_tiles = ((a.own_end + 127) / 128 - a.tile_r0) * a.kb_atoms;
   const int64_t cap = int64_t(dev->sms) * dev->quant_ctas_per_sm;
   const int grid = static_cast<int>(a.n_tiles < cap ? a.n_tiles : cap);
-  quantize_kernel<<<grid, kQThreads, kQSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(tmX, a);
-  return launch_status();
+  return launch_pdl(quantize_kernel, dim3(grid), dim3(kQThreads), kQSmemBytes, reinterpret_cast<cudaStream_t>(stream), 1,
+                    tmX, a);
 }
 
 nvfp4_status_t nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, const float *gs,
@@ -429,24 +457,11 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (!pair) {
     const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
-    gemm_kernel<<<grid, NUM_THREADS, Plan1::BYTES, st>>>(tmA, tmB, p);
-    return launch_status();
+    return launch_pdl(gemm_kernel, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p);
   }
   const int64_t clusters = tiles < dev->gemm2_clusters ? tiles : dev->gemm2_clusters;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = Plan2::BYTES;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemm2_kernel, tmA, tmB, tmSFA, tmSFB, p) != cudaSuccess) return NVFP4_ERR_CUDA;
-  return launch_status();
+  return launch_pdl(gemm2_kernel, dim3(static_cast<unsigned>(2 * clusters)), dim3(NUM_THREADS), Plan2::BYTES, st, 2, tmA,
+                    tmB, tmSFA, tmSFB, p);
 }
 
 int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K) {
@@ -527,8 +542,8 @@ nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols, 
   const int64_t want = (a.bytes / 16 + kFoldThreads - 1) / kFoldThreads;
   const int64_t cap = int64_t(dev->sms) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  fold_scales_kernel<<<grid, kFoldThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
-  return launch_status();
+  return launch_pdl(fold_scales_kernel, dim3(grid), dim3(kFoldThreads), 0, reinterpret_cast<cudaStream_t>(stream), 1,
+                    a);
 }
 
 nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *scale_out,
@@ -550,9 +565,8 @@ nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, i
   const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
   const int64_t cap = int64_t(dev->sms) * 8;
   const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
-  amax_kernel<<<grid, kAmaxThreads, 0, s>>>(a);
-  fp8_scale_finalize_kernel<<<1, 1, 0, s>>>(scale_out);
-  return launch_status();
+  if (nvfp4_status_t e = launch_pdl(amax_kernel, dim3(grid), dim3(kAmaxThreads), 0, s, 1, a)) return e;
+  return launch_pdl(fp8_scale_finalize_kernel, dim3(1), dim3(1), 0, s, 1, scale_out);
 }
 
 nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_t tokens, int64_t width,
@@ -582,8 +596,8 @@ nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_
   const int64_t want = (chunks + kKvThreads - 1) / kKvThreads;
   const int64_t cap = int64_t(dev->sms) * 16;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  kv_cache_fp8_kernel<<<grid, kKvThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
-  return launch_status();
+  return launch_pdl(kv_cache_fp8_kernel, dim3(grid), dim3(kKvThreads), 0, reinterpret_cast<cudaStream_t>(stream), 1,
+                    a);
 }
 
 nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int64_t ld_qk, const void *v_bf16,
@@ -627,10 +641,8 @@ nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int6
   // Short sequences (decode: about one token each) stage 16 tokens at a time, which
   // keeps the shared-memory footprint, and so the occupancy, of the state-bound case.
   if (tokens >= 16 * n_seqs)
-    gdn::recurrence_kernel<32><<<grid, gdn::kThreads, sizeof(gdn::Smem<32>), s>>>(a);
-  else
-    gdn::recurrence_kernel<16><<<grid, gdn::kThreads, sizeof(gdn::Smem<16>), s>>>(a);
-  return launch_status();
+    return launch_pdl(gdn::recurrence_kernel<32>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<32>), s, 1, a);
+  return launch_pdl(gdn::recurrence_kernel<16>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<16>), s, 1, a);
 }
 
 nvfp4_status_t nvfp4_get_device_status(int *code) {

@@ -80,6 +80,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
   return false;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched so that it may start while the previous
+// kernel on the stream finishes.  It may set up shared memory, barriers and TMEM
+// before grid_dep_wait(); it must not touch global memory written by earlier work
+// until grid_dep_wait() returned (the predecessor grids completed and their memory
+// is visible).  Without such a launch the wait returns at once.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream begin launching (it still waits for this one).
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------- copies
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
                                             int32_t x, int32_t y) {

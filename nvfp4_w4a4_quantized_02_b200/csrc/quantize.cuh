@@ -45,6 +45,8 @@ __device__ __forceinline__ uint32_t absmax_bits(uint32_t m, const uint4 &v) {
 // Contiguous rows (ld == cols) are one flat vector stream; otherwise each warp takes
 // whole rows.  Four 16-byte loads in flight per thread.
 __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(AmaxArgs a) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   uint32_t m = 0;
   if (a.ld == a.cols) {
@@ -92,6 +94,8 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(AmaxArgs a) {
 
 // gs = fl32(2688 / amax); amax == 0 -> 1.  In place: amax bits in, gs out.
 __global__ void global_scale_finalize_kernel(float *gs) {
+  grid_dep_wait();
+  grid_dep_launch();
   const float amax = *gs;
   *gs = amax == 0.0f ? 1.0f : __fdiv_rn(2688.0f, amax);
 }
@@ -128,13 +132,15 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
   float *inv_tab = reinterpret_cast<float *>(smem + kQInvOff);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kQBarOff);
   const int tid = threadIdx.x;
-  const float gs = __ldg(a.gs);
-  if (tid < 128) inv_tab[tid] = (tid == 0 || tid == 127) ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(tid));
   if (tid == 0) {
     for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
     fence_barrier_init();
     prefetch_tensormap(&tmX);
   }
+  grid_dep_wait();  // gs and the input may come from the previous kernel
+  grid_dep_launch();
+  const float gs = __ldg(a.gs);
+  if (tid < 128) inv_tab[tid] = (tid == 0 || tid == 127) ? 0.0f : __fdiv_rn(gs, e4m3_to_f32(tid));
   __syncthreads();
 
   const int64_t my_n = a.n_tiles > blockIdx.x ? (a.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
