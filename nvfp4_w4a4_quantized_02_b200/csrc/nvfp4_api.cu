@@ -638,11 +638,14 @@ nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int6
   a.out_fp32 = out_kind == NVFP4_OUT_F32;
   const dim3 grid(gdn::kColBlocks, n_value_heads, static_cast<unsigned>(n_seqs));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // Short sequences (decode: about one token each) stage 16 tokens at a time, which
-  // keeps the shared-memory footprint, and so the occupancy, of the state-bound case.
+  // Short sequences stage fewer tokens at a time: a smaller shared-memory footprint,
+  // so more CTAs per SM in the state-bound case, and less staging work spent on the
+  // empty slots of a chunk (decode: one token per sequence uses the 8-token chunk).
   if (tokens >= 16 * n_seqs)
     return launch_pdl(gdn::recurrence_kernel<32>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<32>), s, 1, a);
-  return launch_pdl(gdn::recurrence_kernel<16>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<16>), s, 1, a);
+  if (tokens >= 4 * n_seqs)
+    return launch_pdl(gdn::recurrence_kernel<16>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<16>), s, 1, a);
+  return launch_pdl(gdn::recurrence_kernel<8>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<8>), s, 1, a);
 }
 
 nvfp4_status_t nvfp4_get_device_status(int *code) {
