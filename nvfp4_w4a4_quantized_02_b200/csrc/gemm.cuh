@@ -374,8 +374,14 @@ __device__ __forceinline__ void store_partial(const Params &p, const uint32_t (&
   }
 }
 
+// Barrier over the epilogue warps only (warps 2 .. 2 + NUM_EPI_WARPS - 1).
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * NUM_EPI_WARPS) : "memory");
+}
+
 // Per-CTA epilogue tables: the segments' alphas and, for an NVFP4 output, the
-// 128 possible values of gs_out / e4m3(sf).
+// 128 possible values of gs_out / e4m3(sf).  Written by threads 64 .. 255, all of
+// them epilogue threads of the GEMM kernels.
 template <int STAGES>
 __device__ __forceinline__ void load_segments(const Params &p, Ctrl<STAGES> &c) {
   if (threadIdx.x >= 64 && threadIdx.x < 64 + p.nseg) {
@@ -487,7 +493,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   grid_dep_wait();  // operands, scales and global scales may come from the previous kernel
   grid_dep_launch();
-  load_segments(p, c);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -580,6 +585,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ----------------------------------------------------------- epilogue
+    // The epilogue tables (global scales of the segments and of the output) are read
+    // here, off the prologue: the first loads need not wait for them.
+    load_segments(p, c);
+    epilogue_bar();
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2; // which 128 of the 256 accumulator columns
     uint32_t acc_phase = 0;
@@ -648,7 +657,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   grid_dep_wait();  // operands, scales and global scales may come from the previous kernel
   grid_dep_launch();
-  load_segments(p, c);
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before either signals the other
@@ -726,6 +734,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       copy_scales<STAGES, true>(c, tmem, sSFA, sSFB, my_tiles * p.k_tiles, warp - COPY_WARP);
   } else {
     // ----------------------------------------------------------- epilogue
+    load_segments(p, c);  // off the prologue, as in gemm_kernel
+    epilogue_bar();
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     uint32_t acc_phase = 0;
