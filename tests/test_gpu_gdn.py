@@ -103,6 +103,31 @@ def test_gdn_ragged_sequences(nv, out_dtype, initial):
     assert nv.device_status() == 0
 
 
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("initial", [False, True])
+def test_gdn_chunked_ragged_sequences(nv, out_dtype, initial):
+    """Sequences long enough for the chunked form (64 tokens or more per sequence on
+    average): empty, one token, one short of a chunk, exactly one chunk, and ragged
+    multi-chunk sequences, with strided rows and gates, with and without an initial
+    state."""
+    import torch
+    hk, hv = 2, 4
+    lens = [0, 1, 63, 64, 130, 200]
+    assert sum(lens) >= 64 * len(lens)
+    d = synth.gdn_recurrence_inputs(lens, hk, hv, seed=160, ld=2 * hk * 128 + hv * 128 + 40)
+    q, k, v, g, b, cu = _dev_inputs(d, hk, hv, gate_ld=hv + 5)
+    rng = np.random.default_rng(161)
+    S0 = (0.3 * rng.standard_normal((len(lens), hv, 128, 128))).astype(np.float32)
+    state = torch.from_numpy(S0).cuda() if initial else torch.full(S0.shape, np.nan, device="cuda")
+    out = nv.gdn_recurrence(q, k, v, g, b, cu, state, initial_state=initial, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _oracle(d, hk, hv, S0 if initial else None)
+    T = sum(lens)
+    _check(out.float().cpu().numpy().reshape(T, hv, 128), o_ref, out_dtype == "bf16")
+    _check(state.cpu().numpy().transpose(0, 1, 3, 2), s_ref, False)
+    assert nv.device_status() == 0
+
+
 def test_gdn_decode_batch(nv):
     """Decode: 32 sequences of one token each over a carried state (the short-sequence
     staging path), all 32 value heads over 16 key heads."""
