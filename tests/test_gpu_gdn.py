@@ -105,11 +105,10 @@ def test_gdn_ragged_sequences(nv, out_dtype, initial):
 
 @pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("initial", [False, True])
-def test_gdn_chunked_ragged_sequences(nv, out_dtype, initial):
-    """Sequences long enough for the chunked form (64 tokens or more per sequence on
-    average): empty, one token, one short of a chunk, exactly one chunk, and ragged
-    multi-chunk sequences, with strided rows and gates, with and without an initial
-    state."""
+def test_gdn_long_ragged_sequences(nv, out_dtype, initial):
+    """Long sequences (64 tokens or more per sequence on average, the prefill launch):
+    empty, one token, 63, 64 and ragged multi-chunk sequences across the 32-token
+    staging chunks, with strided rows and gates, with and without an initial state."""
     import torch
     hk, hv = 2, 4
     lens = [0, 1, 63, 64, 130, 200]
