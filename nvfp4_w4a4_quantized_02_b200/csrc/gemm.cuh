@@ -466,6 +466,11 @@ __device__ __forceinline__ void init_barriers(Ctrl<STAGES> &c, uint32_t acc_empt
 }
 
 // ============================================================ 1-CTA kernel
+// kPartial: the split-K form, whose epilogue only stores the raw FP32 sums (the
+// epilogue of the linear runs in splitk_epilogue_kernel).  A separate instantiation
+// keeps its code small: a decode-size launch spends much of its few microseconds
+// fetching instructions.
+template <bool kPartial>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ Params p) {
@@ -586,13 +591,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ----------------------------------------------------------- epilogue
     // The epilogue tables (global scales of the segments and of the output) are read
-    // here, off the prologue: the first loads need not wait for them.
-    load_segments(p, c);
-    epilogue_bar();
+    // here, off the prologue: the first loads need not wait for them.  (The split-K
+    // form stores raw sums and needs none.)
+    if constexpr (!kPartial) {
+      load_segments(p, c);
+      epilogue_bar();
+    }
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2; // which 128 of the 256 accumulator columns
     uint32_t acc_phase = 0;
-    const float gs_out = p.out_kind == OUT_NVFP4 ? __ldg(p.gs_out) : 1.0f;
+    const float gs_out = !kPartial && p.out_kind == OUT_NVFP4 ? __ldg(p.gs_out) : 1.0f;
     for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
       int tile, split, k0, k1, mt, nt;
       unit_coords(p, u, tile, split, k0, k1);
@@ -606,7 +614,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.acc_empty);
       const int row = mt * BM + 32 * q + lane;
-      if (p.partial) {
+      if constexpr (kPartial) {
         store_partial(p, v, split, row, nt * BN + half * 128);
       } else {
         epilogue_row(p, c, v, row, nt, half, gs_out);

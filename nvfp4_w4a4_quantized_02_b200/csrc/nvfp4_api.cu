@@ -52,7 +52,9 @@ nvfp4_status_t current_device(DeviceInfo **info) {
   }
   if (!d.ok) return NVFP4_ERR_UNSUPPORTED_DEVICE;
   if (!d.attrs) {
-    if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm::gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::Plan1::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::Plan1::BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::Plan2::BYTES) != cudaSuccess ||
@@ -312,7 +314,7 @@ nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvf
   const int64_t units = int64_t(p.m_tiles) * p.n_tiles * p.splits;
   if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
-  if (nvfp4_status_t e = launch_pdl(gemm_kernel, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p))
+  if (nvfp4_status_t e = launch_pdl(gemm_kernel<true>, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p))
     return e;
   const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (p.M + 127) / 128 * 128 : p.M;
   const int64_t threads = rows_cover * (p.Nout / 16);  // one thread per 16-column block
@@ -453,7 +455,7 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (!pair) {
     const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
-    return launch_pdl(gemm_kernel, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p);
+    return launch_pdl(gemm_kernel<false>, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p);
   }
   const int64_t clusters = tiles < dev->gemm2_clusters ? tiles : dev->gemm2_clusters;
   return launch_pdl(gemm2_kernel, dim3(static_cast<unsigned>(2 * clusters)), dim3(NUM_THREADS), Plan2::BYTES, st, 2, tmA,
