@@ -193,11 +193,15 @@ NVFP4_API nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_
  *   and applies exactly the epilogue and output kind of nvfp4_linear (per-segment
  *   alpha, SiLU*mul or GDN gates, BF16 / FP32 / NVFP4 store).  Results equal
  *   nvfp4_linear's up to the order of the FP32 additions.
+ *   Up to 64 token rows (M <= 64) a unit is 128 weight rows x all tokens x its K
+ *   range, computed with the weight as the MMA's 128-row operand and the tokens
+ *   (padded to 32 or 64) as its N; above 64 rows it is an output tile of 128 x 256.
  *   Source: the blog's results section (結果: decode at concurrency 32, 1,154 tok/s
  *   against 621 tok/s in BF16) is the regime; the method is nvfp4_linear's.
  *   Arguments as nvfp4_linear, plus:
  *   split_k: 1 .. K/256 (nvfp4_splitk_default gives the library's choice); with 1
- *   the call runs nvfp4_linear itself and does not touch the workspace;
+ *   and M > 64 the call runs nvfp4_linear itself and does not touch the workspace
+ *   (with M <= 64 one split still goes through the workspace and the second kernel);
  *   workspace: device, >= nvfp4_splitk_workspace_bytes(M, N, split_k) bytes,
  *   16-byte aligned, owned by the caller; its contents on entry do not matter and
  *   are overwritten.  Two calls that share a workspace must not overlap on the GPU.
@@ -215,10 +219,10 @@ NVFP4_API nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const flo
 NVFP4_API size_t nvfp4_splitk_workspace_bytes(int64_t M, int64_t N, int split_k);
 
 /* The split count the library would choose for an M x N x K linear on the current
- * device (>= 1, <= K/256): as many splits as keep all (output tile of 128 x 256, K
- * range) work units in one wave on the SMs, i.e. SMs / tiles rounded down, with at
- * least 4 K tiles of 256 per split.  0 for invalid sizes or when the device cannot be
- * queried. */
+ * device (>= 1, <= K/256): as many splits as keep all (tile, K range) work units in
+ * one wave on the SMs, i.e. SMs / tiles rounded down, with at least 4 K tiles of 256
+ * per split.  A tile is 128 weight rows for M <= 64 and 128 x 256 outputs above.  0
+ * for invalid sizes or when the device cannot be queried. */
 NVFP4_API int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K);
 
 /*

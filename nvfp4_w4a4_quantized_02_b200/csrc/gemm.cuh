@@ -124,6 +124,8 @@ struct Params {
   const float *gs_out;
   uint8_t *out_scales;
   int64_t out_kb_atoms;
+  // decode kernel: token rows per MMA (32 or 64)
+  int dn;
 };
 
 template <int STAGES>
@@ -769,6 +771,223 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   cluster_sync();  // neither CTA leaves while the other may still signal it
   tc_fence_after();
   if (warp == 1) tmem_dealloc_cg2(tmem, TMEM_COLS);
+}
+
+// ======================================================== decode kernel
+// The decode regime (a few token rows against a large weight) with the operands'
+// roles swapped: 128 weight rows are the MMA's M and the DN (32 or 64) token rows its
+// N, so no MMA row is padding and a stage carries a 16 KB weight tile, a small token
+// tile and two scale sets of 4 atoms each (8 copies, against 12 for a 128 x 256 tile).
+// Seven stages stay in flight to keep HBM busy while the weights stream through.
+// Work units are (128-row weight tile, K range); each writes its raw FP32 sums to
+// partial[split][m][n] (n = weight row = output column), and splitk_epilogue_kernel
+// applies the epilogue of the linear, as for the split-K form of gemm_kernel.
+// Accumulator: TMEM lane = weight row, column = token.  B's scales (the tokens'): row
+// 32c + i at lane 32q + i, column base + c, c < DN / 32, all inside one atom copy.
+constexpr int DEC_BM = 128;              // weight rows per tile (MMA M)
+constexpr int DEC_DN_MAX = 64;           // token rows per MMA (N)
+constexpr int DEC_STAGES = 7;
+constexpr int DEC_W_BYTES = DEC_BM * BK / 2;       // 16 KB
+constexpr int DEC_X_BYTES = DEC_DN_MAX * BK / 2;   // 8 KB
+constexpr int DEC_SF_BYTES = 4 * SF_ATOM;          // 2 KB: 4 k-steps of one 128-row group
+constexpr int DEC_THREADS = 256;                   // producer, MMA, 4 epilogue, 2 copier warps
+constexpr int DEC_EPI_WARP = 2;
+constexpr int DEC_COPY_WARP = 6;
+constexpr uint32_t DEC_ACC_COL = 0;                // DEC_DN_MAX FP32 columns
+constexpr uint32_t DEC_SF_COL = DEC_DN_MAX;        // then one 32-column scale set per stage
+__host__ __device__ constexpr uint32_t dec_sfw_col(int stage) { return DEC_SF_COL + 32 * stage; }
+__host__ __device__ constexpr uint32_t dec_sfx_col(int stage) { return DEC_SF_COL + 32 * stage + 16; }
+static_assert(dec_sfx_col(DEC_STAGES - 1) + 16 <= TMEM_COLS, "TMEM columns");
+
+struct PlanD {
+  static constexpr int CTRL_BYTES = 1024;
+  static constexpr int W_OFF = CTRL_BYTES;
+  static constexpr int X_OFF = W_OFF + DEC_STAGES * DEC_W_BYTES;
+  static constexpr int SFW_OFF = X_OFF + DEC_STAGES * DEC_X_BYTES;
+  static constexpr int SFX_OFF = SFW_OFF + DEC_STAGES * DEC_SF_BYTES;
+  static constexpr int END = SFX_OFF + DEC_STAGES * DEC_SF_BYTES;
+  static constexpr int BYTES = END + 1024;  // slack to align the base to 1024
+};
+static_assert(PlanD::BYTES <= 227 * 1024, "shared memory");
+
+struct CtrlD {
+  uint64_t full[DEC_STAGES];
+  uint64_t empty[DEC_STAGES];
+  uint64_t sf_ready[DEC_STAGES];
+  uint64_t acc_full;
+  uint64_t acc_empty;
+  uint64_t drain;
+  uint64_t sf_drain[2];
+  uint32_t tmem_base;
+};
+static_assert(sizeof(CtrlD) <= PlanD::CTRL_BYTES, "control block too large");
+
+// tmW: weight codes, boxes of 128 rows; tmX: token codes, boxes of p.dn rows.
+// p.sfb: the weight's scales, p.sfa: the tokens' (one 128-row group: p.M <= 64).
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                  const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  CtrlD &c = *reinterpret_cast<CtrlD *>(smem);
+  uint8_t *sW = smem + PlanD::W_OFF;
+  uint8_t *sX = smem + PlanD::X_OFF;
+  uint8_t *sSFW = smem + PlanD::SFW_OFF;
+  uint8_t *sSFX = smem + PlanD::SFX_OFF;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DEC_STAGES; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+      mbar_init(&c.sf_ready[s], 2);
+    }
+    mbar_init(&c.acc_full, 1);
+    mbar_init(&c.acc_empty, 4);
+    mbar_init(&c.drain, 1);
+    mbar_init(&c.sf_drain[0], 1);
+    mbar_init(&c.sf_drain[1], 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  grid_dep_wait();  // the tokens' codes and scales may come from the previous kernel
+  grid_dep_launch();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  const int num_units = p.n_tiles * p.splits;
+  const uint32_t x_bytes = static_cast<uint32_t>(p.dn) * (BK / 2);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        int nt, split, k0, k1;
+        unit_coords(p, u, nt, split, k0, k1);
+        const uint8_t *sfw_src = p.sfb + ((int64_t)nt * p.kb_atoms) * SF_ATOM;
+        for (int kt = k0; kt < k1; ++kt) {
+          if (!mbar_wait(&c.empty[stage], phase ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&c.full[stage], DEC_W_BYTES + x_bytes + 2 * DEC_SF_BYTES);
+          const int kx = kt * (BK / 2);
+          tma_load_2d(sW + stage * DEC_W_BYTES, &tmW, &c.full[stage], kx, nt * DEC_BM);
+          tma_load_2d(sX + stage * DEC_X_BYTES, &tmX, &c.full[stage], kx, 0);
+          bulk_load(sSFW + stage * DEC_SF_BYTES, sfw_src + (int64_t)kt * DEC_SF_BYTES, DEC_SF_BYTES, &c.full[stage]);
+          bulk_load(sSFX + stage * DEC_SF_BYTES, p.sfa + (int64_t)kt * DEC_SF_BYTES, DEC_SF_BYTES, &c.full[stage]);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == DEC_STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // let every copy this thread issued land before the CTA can exit
+      for (int s = 0; s < DEC_STAGES; ++s)
+        if (armed & (1u << s)) mbar_wait(&c.full[s], (armed_phase >> s) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(DEC_BM, p.dn);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        int nt, split, k0, k1;
+        unit_coords(p, u, nt, split, k0, k1);
+        if (!mbar_wait(&c.acc_empty, acc_phase ^ 1)) break;
+        acc_phase ^= 1;
+        tc_fence_after();
+        for (int kt = k0; kt < k1; ++kt) {
+          if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t w_desc = sdesc_sw128_kmajor(smem_u32(sW + stage * DEC_W_BYTES));
+          const uint64_t x_desc = sdesc_sw128_kmajor(smem_u32(sX + stage * DEC_X_BYTES));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_nvfp4(tmem + DEC_ACC_COL, w_desc + 2 * j, x_desc + 2 * j, idesc, tmem + dec_sfw_col(stage) + 4 * j,
+                      tmem + dec_sfx_col(stage) + 4 * j, (kt != k0) | (j != 0));
+          tc_commit(&c.empty[stage]);
+          if (++stage == DEC_STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (ok) tc_commit(&c.acc_full);
+      }
+      tc_commit(&c.drain);
+      mbar_wait(&c.drain, 0);
+    }
+  } else if (warp >= DEC_COPY_WARP) {
+    // ---------------------------------------------------------- scale copiers
+    // Part 0: the weight's 4 atoms of the stage; part 1: the tokens' 4 atoms.
+    if (lane == 0) {
+      const int part = warp - DEC_COPY_WARP;
+      int total = 0;
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        int nt, split, k0, k1;
+        unit_coords(p, u, nt, split, k0, k1);
+        total += k1 - k0;
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int g = 0; g < total; ++g) {
+        if (!mbar_wait(&c.full[stage], phase)) break;
+        tc_fence_after();
+        const uint32_t src = smem_u32((part == 0 ? sSFW : sSFX) + stage * DEC_SF_BYTES);
+        const uint32_t col = part == 0 ? dec_sfw_col(stage) : dec_sfx_col(stage);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cp_scale_atom<false>(tmem + col + 4 * j, src + j * SF_ATOM);
+        tc_commit(&c.sf_ready[stage]);
+        if (++stage == DEC_STAGES) { stage = 0; phase ^= 1; }
+      }
+      tc_commit(&c.sf_drain[part]);
+      mbar_wait(&c.sf_drain[part], 0);
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    // Warps 2..5: TMEM lane quadrant q = warp % 4, lane = weight row 32 q + lane of the
+    // tile, one column per token.
+    const int q = warp & 3;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      int nt, split, k0, k1;
+      unit_coords(p, u, nt, split, k0, k1);
+      if (!mbar_wait(&c.acc_full, acc_phase)) break;
+      acc_phase ^= 1;
+      tc_fence_after();
+      uint32_t v[2][32];
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16) + DEC_ACC_COL;
+      tmem_ld_32x32b_x32(lane_addr, v[0]);
+      if (p.dn > 32) tmem_ld_32x32b_x32(lane_addr + 32, v[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.acc_empty);
+      const int n = nt * DEC_BM + 32 * q + lane;
+      if (n < p.N) {
+        float *dst = p.partial + (int64_t)split * p.M * p.N + n;
+#pragma unroll
+        for (int m = 0; m < 32; ++m)
+          if (m < p.M) dst[(int64_t)m * p.N] = __uint_as_float(v[0][m]);
+        if (p.dn > 32) {
+#pragma unroll
+          for (int m = 0; m < 32; ++m)
+            if (32 + m < p.M) dst[(int64_t)(32 + m) * p.N] = __uint_as_float(v[1][m]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // ======================================================= split-K epilogue

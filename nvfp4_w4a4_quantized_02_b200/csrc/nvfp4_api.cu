@@ -58,6 +58,8 @@ nvfp4_status_t current_device(DeviceInfo **info) {
                              gemm::Plan1::BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::Plan2::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::PlanD::BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
             cudaSuccess ||
         cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes) !=
@@ -110,15 +112,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map of packed codes [rows x K/2] bytes: 128-byte x 128-row boxes with the
+// Tensor map of packed codes [rows x K/2] bytes: 128-byte x box_rows boxes with the
 // 128-byte swizzle (the smem layout the MMA descriptors describe); rows beyond
 // `rows` read as zero.
-bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K) {
+bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, unsigned box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  cuuint32_t box[2] = {128, 128};
+  cuuint32_t box[2] = {128, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -286,12 +288,13 @@ nvfp4_status_t prepare_linear(const nvfp4_operand_t *A, const float *gs_a, const
 
 // Split count of the split-K linear: as many splits as keep all work units in one
 // wave on the SMs (SMs / tiles, rounded down), with at least 4 K tiles (1024 K) per
-// split.  Measured on the 496-linear decode step at 32 rows (one CUDA graph per step):
-// about 6 ms with a one-wave fill against 7.3-7.5 ms when only the 17408-long down
-// projection was split; a second wave (the MLP gate|up, 136 tiles, split twice) cost
-// 29 instead of 24 us per launch, and 2 K tiles per split was slower again.
+// split.  Tiles are 128 weight rows for the decode kernel (M <= 64), else 128 x 256.
+// On the decode kernel at 32 rows the rule picks the fastest of splits 1, 2, 3, 4, 6
+// for five of the six shapes of the 496-linear decode step; for the 12352-row GDN
+// in-projection it picks 1 (13.2 us), where 3 measured 12.8 us.
 int default_splits(int64_t M, int64_t N, int64_t K, int sms) {
-  const int64_t tiles = (M + gemm::BM - 1) / gemm::BM * ((N + gemm::BN - 1) / gemm::BN);
+  const int64_t tiles = M <= gemm::DEC_DN_MAX ? (N + gemm::DEC_BM - 1) / gemm::DEC_BM
+                                               : (M + gemm::BM - 1) / gemm::BM * ((N + gemm::BN - 1) / gemm::BN);
   const int64_t k_tiles = K / gemm::BK;
   int64_t s = sms / tiles;
   if (s > k_tiles / 4) s = k_tiles / 4;
@@ -303,19 +306,33 @@ int default_splits(int64_t M, int64_t N, int64_t K, int sms) {
 nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvfp4_operand_t *W, int splits,
                              float *workspace, const DeviceInfo *dev, cudaStream_t st) {
   using namespace gemm;
-  CUtensorMap tmA, tmB;
-  if (!make_codes_map(&tmA, A->codes, p.M, p.K) || !make_codes_map(&tmB, W->codes, p.N, p.K)) return NVFP4_ERR_CUDA;
   p.kt_per_split = (p.k_tiles + splits - 1) / splits;
   p.splits = (p.k_tiles + p.kt_per_split - 1) / p.kt_per_split;  // no empty split
   p.partial = workspace;
   p.tile_mode = MODE_NONE;
-  p.m_tiles = (p.M + BM - 1) / BM;
-  p.n_tiles = (p.N + BN - 1) / BN;
-  const int64_t units = int64_t(p.m_tiles) * p.n_tiles * p.splits;
-  if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
-  if (nvfp4_status_t e = launch_pdl(gemm_kernel<true>, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p))
-    return e;
+  CUtensorMap tmA, tmB;
+  if (p.M <= DEC_DN_MAX) {  // decode size: weight rows are the MMA's M, tokens its N
+    p.dn = p.M <= 32 ? 32 : DEC_DN_MAX;
+    p.m_tiles = 1;
+    p.n_tiles = (p.N + DEC_BM - 1) / DEC_BM;
+    if (!make_codes_map(&tmB, W->codes, p.N, p.K) || !make_codes_map(&tmA, A->codes, p.M, p.K, p.dn))
+      return NVFP4_ERR_CUDA;
+    const int64_t units = int64_t(p.n_tiles) * p.splits;
+    if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
+    if (nvfp4_status_t e = launch_pdl(decode_kernel, dim3(grid), dim3(DEC_THREADS), PlanD::BYTES, st, 1, tmB, tmA, p))
+      return e;
+  } else {
+    if (!make_codes_map(&tmA, A->codes, p.M, p.K) || !make_codes_map(&tmB, W->codes, p.N, p.K)) return NVFP4_ERR_CUDA;
+    p.m_tiles = (p.M + BM - 1) / BM;
+    p.n_tiles = (p.N + BN - 1) / BN;
+    const int64_t units = int64_t(p.m_tiles) * p.n_tiles * p.splits;
+    if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
+    if (nvfp4_status_t e =
+            launch_pdl(gemm_kernel<true>, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p))
+      return e;
+  }
   const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (p.M + 127) / 128 * 128 : p.M;
   const int64_t threads = rows_cover * (p.Nout / 16);  // one thread per 16-column block
   const int64_t blocks = (threads + REDUCE_THREADS - 1) / REDUCE_THREADS;
@@ -485,7 +502,10 @@ nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const float *gs_a, 
   if (!workspace) return NVFP4_ERR_INVALID_ARG;
   if (workspace_bytes < nvfp4_splitk_workspace_bytes(p.M, p.N, split_k)) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return NVFP4_ERR_MISALIGNED;
-  if (split_k == 1)  // one split: the ordinary kernel, without partials or the second kernel
+  // One split above decode size: the ordinary kernel, without partials or the second
+  // kernel.  Up to 64 rows the decode kernel and the reduction beat it even unsplit
+  // (a 496-linear decode step at 32 rows: 4.74 ms against 6.86 ms).
+  if (split_k == 1 && p.M > DEC_DN_MAX)
     return nvfp4_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, stream);
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;

@@ -39,14 +39,15 @@ def test_down_proj_decode_full_size(nv):
     w = nv.quantize(to_dev_bf16(wb))
     s_def = nv.splitk_default(M, N, K)
     assert 1 < s_def <= K // 256  # 20 output tiles, 68 K tiles: the split pays here
-    # the rule: SMs // tiles splits (one wave of work units), with >= 4 K tiles per split
+    # the rule: SMs // tiles splits (one wave of work units), with >= 4 K tiles per split;
+    # up to 64 rows a tile is 128 weight rows (all tokens), else 128 x 256 outputs
     sms = torch.cuda.get_device_properties(0).multi_processor_count
 
     def rule(m, n, k):
-        tiles = -(-m // 128) * -(-n // 256)
+        tiles = -(-n // 128) if m <= 64 else -(-m // 128) * -(-n // 256)
         return max(1, min(k // 256 // 4, sms // tiles))
     for shape in [(M, N, K), (M, 34816, 5120), (M, 5120, 4096), (M, 12352, 5120), (4096, 5120, 4096),
-                  (M, 1024, 512)]:
+                  (M, 1024, 512), (64, 5120, 5120), (65, 5120, 5120)]:
         assert nv.splitk_default(*shape) == rule(*shape), shape
     for s in (s_def, 1, 5):
         y32 = nv.linear_splitk(a, w, out_dtype="f32", split_k=s)
@@ -62,9 +63,11 @@ def test_down_proj_decode_full_size(nv):
     assert nv.device_status() == 0
 
 
-@pytest.mark.parametrize("M", [1, 7, 100, 129, 200])
+@pytest.mark.parametrize("M", [1, 7, 32, 33, 64, 65, 100, 129, 200])
 def test_ragged_rows_and_splits(nv, M):
-    """Rows that fill part of a 128-row tile, or span two; every split count."""
+    """Rows that fill part of a 128-row tile, or span two; every split count.  Up to
+    64 rows the decode kernel runs (32 or 64 token columns per MMA), above it the
+    128 x 256 tile kernel; 400 weight rows end in a ragged 128-row weight tile."""
     K, segs = 768, [("s0", 128), ("s1", 176), ("s2", 96)]
     ws = synth.segmented_weights(segs, K, seed=50, multipliers={"s0": 1.0, "s1": 5.0, "s2": 0.25})
     xb = synth.outlier_activations(M, K, seed=51)
