@@ -27,7 +27,8 @@ def _sync():
 
 def test_down_proj_decode_full_size(nv):
     """32 decode tokens through the MLP down projection (5120 x 17408): FP32 and BF16
-    outputs against the oracle, with the library's split count and with splits 1 and 5."""
+    outputs against the oracle, with the library's split count and with splits 1, 5
+    and 10."""
     import torch
     M, N, K = 32, 5120, 17408
     xb = synth.student_t_activations(M, K, seed=40)
@@ -49,7 +50,7 @@ def test_down_proj_decode_full_size(nv):
     for shape in [(M, N, K), (M, 34816, 5120), (M, 5120, 4096), (M, 12352, 5120), (4096, 5120, 4096),
                   (M, 1024, 512), (64, 5120, 5120), (65, 5120, 5120)]:
         assert nv.splitk_default(*shape) == rule(*shape), shape
-    for s in (s_def, 1, 5):
+    for s in (s_def, 1, 5, 10):
         y32 = nv.linear_splitk(a, w, out_dtype="f32", split_k=s)
         y16 = nv.linear_splitk(a, w, out_dtype="bf16", split_k=s)
         _sync()
@@ -86,9 +87,10 @@ def test_ragged_rows_and_splits(nv, M):
         assert rel_fro(y.cpu().numpy(), ref) <= 1e-3, (M, s)
 
 
-def test_gdn_inproj_decode_full_size(nv):
+@pytest.mark.parametrize("split_k", [None, 3])
+def test_gdn_inproj_decode_full_size(nv, split_k):
     """32 decode tokens through the fused GDN in-projection (12352 x 5120, six
-    segments) with the gate epilogue."""
+    segments) with the gate epilogue: the library's split count and 3 splits."""
     import torch
     M, K = 32, 5120
     xb = synth.outlier_activations(M, K, seed=60)
@@ -110,16 +112,19 @@ def test_gdn_inproj_decode_full_size(nv):
     g = torch.empty((M, 32), dtype=torch.float32, device="cuda")
     gates = dict(beta_begin=N - 64, alpha_begin=N - 32, n_heads=32, A_log=to_dev_f32(a_log),
                  dt_bias=to_dev_f32(dt_bias), beta_out=beta, g_out=g)
-    out = nv.linear_splitk(a, w, segments=dsegs, epilogue="gdn_gates", gates=gates, out_dtype="bf16")
+    out = nv.linear_splitk(a, w, segments=dsegs, epilogue="gdn_gates", gates=gates, out_dtype="bf16",
+                           split_k=split_k)
     _sync()
     assert np.max(np.abs(beta.cpu().numpy() - beta_ref)) <= 1e-3
     assert np.max(np.abs(g.cpu().numpy() - g_ref)) <= 1e-3
     assert_gemm_close(out[:, :N - 64], y[:, :N - 64])
 
 
-def test_silu_mul_requant_decode(nv):
+@pytest.mark.parametrize("split_k", [1, 3, 4])
+def test_silu_mul_requant_decode(nv, split_k):
     """Gate|up with SiLU*mul and NVFP4 re-quantisation: BF16 output against the oracle;
-    the NVFP4 output equals the standalone quantiser applied to the BF16 output."""
+    the NVFP4 output equals the standalone quantiser applied to the BF16 output.  With
+    4 K tiles, splits 1, 3 (two K ranges of 2, so 2 splits) and 4."""
     import torch
     M, K, Nh = 32, 1024, 2048
     ws = synth.segmented_weights([("gate", Nh), ("up", Nh)], K, seed=70, multipliers={"gate": 1, "up": 2})
@@ -134,13 +139,13 @@ def test_silu_mul_requant_decode(nv):
     h_ref = oracle.silu_mul(y[:, :Nh], y[:, Nh:])
     w, dsegs = nv.quantize_fused([to_dev_bf16(wb) for _, wb in ws])
     a = nv.quantize(to_dev_bf16(xb))
-    h16 = nv.linear_splitk(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="bf16", split_k=3)
+    h16 = nv.linear_splitk(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="bf16", split_k=split_k)
     _sync()
     assert_gemm_close(h16, h_ref)
     gs_h = nv.global_scale(h16)
     scales = torch.full((nv.scale_bytes(M, Nh),), 0xAB, dtype=torch.uint8, device="cuda")
     hq = nv.linear_splitk(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=gs_h,
-                          out_scales=scales, split_k=3)
+                          out_scales=scales, split_k=split_k)
     hq2 = nv.quantize(h16, gs_h)
     _sync()
     assert torch.equal(hq.codes, hq2.codes) and torch.equal(hq.scales, hq2.scales)
