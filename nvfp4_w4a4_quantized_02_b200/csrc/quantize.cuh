@@ -16,6 +16,12 @@
 // word into a shared atom, which 32 threads then write out as 512 contiguous
 // bytes.  gs / e4m3(sf) takes one of 127 values per call: it is tabulated once
 // per CTA (the same FP32 division, so bit-identical).
+//
+// Two stages per CTA with four CTAs per SM (the register limit at 256 threads)
+// streamed fastest: 0.84 of the measured copy bandwidth at 32768 x 5120 against 0.79
+// with four stages and 0.70 with six.  More tiles in flight per CTA spread the
+// concurrent reads over more DRAM rows.  The codes and scales are stored with the
+// default L2 policy (not evict-first): the GEMM that consumes them usually runs next.
 #pragma once
 
 #include "quant_math.cuh"
@@ -104,7 +110,7 @@ __global__ void global_scale_finalize_kernel(float *gs) {
 constexpr int kQThreads = 256;
 constexpr int kQTileRows = 128;
 constexpr int kQTileCols = 64;
-constexpr int kQStages = 4;
+constexpr int kQStages = 2;
 constexpr int kQTileBytes = kQTileRows * kQTileCols * 2;  // 16 KB of BF16
 constexpr int kQAtomOff = kQStages * kQTileBytes;         // 512-byte scale atom
 constexpr int kQInvOff = kQAtomOff + 512;                 // 128 floats: gs / e4m3(sf)
@@ -208,13 +214,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
       uint8_t *dst = a.codes + dest * a.code_ld + col / 2;
       if (col + 32 <= a.cols) {
         if (vec16) {
-          __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(code[0], code[1], code[2], code[3]));
+          __stcg(reinterpret_cast<uint4 *>(dst), make_uint4(code[0], code[1], code[2], code[3]));
         } else {
-          __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(code[0], code[1]));
-          __stcs(reinterpret_cast<uint2 *>(dst + 8), make_uint2(code[2], code[3]));
+          __stcg(reinterpret_cast<uint2 *>(dst), make_uint2(code[0], code[1]));
+          __stcg(reinterpret_cast<uint2 *>(dst + 8), make_uint2(code[2], code[3]));
         }
       } else {
-        __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(code[0], code[1]));  // cols % 16 == 0: one block left
+        __stcg(reinterpret_cast<uint2 *>(dst), make_uint2(code[0], code[1]));  // cols % 16 == 0: one block left
       }
     }
     // scale word of row rho: blocks 0,1 from thread 2*rho, blocks 2,3 from thread 2*rho+1
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
       __syncthreads();
       if (tid < 32) {
         uint4 *dst = reinterpret_cast<uint4 *>(a.scales + (rt * a.kb_atoms + ka) * 512);
-        __stcs(dst + tid, reinterpret_cast<const uint4 *>(atom)[tid]);
+        __stcg(dst + tid, reinterpret_cast<const uint4 *>(atom)[tid]);
       }
     } else if (h == 0 && own) {
       *reinterpret_cast<uint32_t *>(a.scales + scale_word_offset(dest, ka, a.kb_atoms)) = word;
