@@ -407,7 +407,7 @@ nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols
   a.amax_bits = reinterpret_cast<unsigned int *>(gs_out);
   const int64_t vecs = rows * (cols / 8);
   const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
-  const int64_t cap = int64_t(dev->sms) * 8;
+  const int64_t cap = int64_t(dev->sms) * 4;
   const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
   if (nvfp4_status_t e = launch_pdl(amax_kernel, dim3(grid), dim3(kAmaxThreads), 0, s, 1, a)) return e;
   return launch_pdl(global_scale_finalize_kernel, dim3(1), dim3(1), 0, s, 1, gs_out);
@@ -581,7 +581,7 @@ nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, i
   a.amax_bits = reinterpret_cast<unsigned int *>(scale_out);
   const int64_t vecs = rows * (cols / 8);
   const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
-  const int64_t cap = int64_t(dev->sms) * 8;
+  const int64_t cap = int64_t(dev->sms) * 4;
   const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
   if (nvfp4_status_t e = launch_pdl(amax_kernel, dim3(grid), dim3(kAmaxThreads), 0, s, 1, a)) return e;
   return launch_pdl(fp8_scale_finalize_kernel, dim3(1), dim3(1), 0, s, 1, scale_out);

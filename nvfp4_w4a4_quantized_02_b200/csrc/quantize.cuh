@@ -19,8 +19,8 @@
 //
 // Two stages per CTA with four CTAs per SM (the register limit at 256 threads)
 // streamed fastest: 0.84 of the measured copy bandwidth at 32768 x 5120 against 0.79
-// with four stages and 0.70 with six.  More tiles in flight per CTA spread the
-// concurrent reads over more DRAM rows.  The codes and scales are stored with the
+// with four stages and 0.70 with six (more tiles in flight per CTA presumably spread
+// the concurrent reads over more DRAM rows).  The codes and scales are stored with the
 // default L2 policy (not evict-first): the GEMM that consumes them usually runs next.
 #pragma once
 
@@ -48,8 +48,8 @@ __device__ __forceinline__ uint32_t absmax_bits(uint32_t m, const uint4 &v) {
 }
 
 // max over |x| of the BF16 bit patterns (order-preserving for non-negative values).
-// Contiguous rows (ld == cols) are one flat vector stream; otherwise each warp takes
-// whole rows.  Four 16-byte loads in flight per thread.
+// Contiguous rows (ld == cols) are one flat vector stream with eight 16-byte loads in
+// flight per thread; otherwise each warp takes whole rows, four loads at a time.
 __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(AmaxArgs a) {
   grid_dep_wait();
   grid_dep_launch();
@@ -60,12 +60,12 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(AmaxArgs a) {
     const int64_t n = a.rows * a.cols / 8;
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
     int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; v + 3 * T < n; v += 4 * T) {
-      uint4 q[4];
+    for (; v + 7 * T < n; v += 8 * T) {
+      uint4 q[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) q[i] = __ldcs(x + v + i * T);
+      for (int i = 0; i < 8; ++i) q[i] = __ldcs(x + v + i * T);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) m = absmax_bits(m, q[i]);
+      for (int i = 0; i < 8; ++i) m = absmax_bits(m, q[i]);
     }
     for (; v < n; v += T) m = absmax_bits(m, __ldcs(x + v));
   } else {
