@@ -862,7 +862,7 @@ class GDNRecurrence(Workload):
     Algorithmic FLOPs per token and value head: 7 d_k d_v (prediction S^T k 2, decay 1,
     rank-1 write 2, read-out S^T q 2)."""
     unit = "TFLOP/s"
-    dtype = "fp32 state and arithmetic (bf16 q/k/v/out)"
+    dtype = "fp32 state; bf16 tensor-core products, fp32 operands split hi/lo (bf16 q/k/v/out)"
     SEQ = 4096
 
     def __init__(self, nv, M=8192, seed=0):
@@ -877,7 +877,9 @@ class GDNRecurrence(Workload):
         self.launches_per_step = 1
         self.l2_note = (f"inputs larger than L2 (q|k|v rows {M * 8192 * 2 / 1e6:.0f} MB, out "
                         f"{M * 4096 * 2 / 1e6:.0f} MB)")
-        self.dominant = ("gdn_recurrence", self.flops, "alu", "gdn recurrence_kernel<32> (state in registers)")
+        self.dominant = ("gdn_recurrence", self.flops, "alu",
+                         "gdn chunk_kernel (64-token chunks; products on BF16 mma.sync with FP32 operands split "
+                         "hi/lo; rate in the token recurrence's FLOPs)")
         self.phases = {"gdn_recurrence": ("ALU", self.flops)}
         torch.cuda.synchronize()
 

@@ -13,6 +13,7 @@
 #include "fold.cuh"
 #include "kvcache.cuh"
 #include "gdn.cuh"
+#include "gdn_chunk.cuh"
 
 using namespace nvfp4;
 
@@ -67,7 +68,9 @@ nvfp4_status_t current_device(DeviceInfo **info) {
         cudaFuncSetAttribute(gdn::recurrence_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(sizeof(gdn::Smem<32>))) != cudaSuccess ||
         cudaFuncSetAttribute(gdn::recurrence_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(sizeof(gdn::Smem<16>))) != cudaSuccess)
+                             int(sizeof(gdn::Smem<16>))) != cudaSuccess ||
+        cudaFuncSetAttribute(gdn::chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(sizeof(gdn::ChunkSmem))) != cudaSuccess)
       return NVFP4_ERR_CUDA;
     {
       cudaLaunchConfig_t cfg = {};
@@ -656,6 +659,10 @@ nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int6
   a.out_fp32 = out_kind == NVFP4_OUT_F32;
   const dim3 grid(gdn::kColBlocks, n_value_heads, static_cast<unsigned>(n_seqs));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // Long sequences (prefill): the chunked form on the tensor cores.
+  if (tokens >= 64 * n_seqs)
+    return launch_pdl(gdn::chunk_kernel, dim3(gdn::kChunkColBlocks, n_value_heads, static_cast<unsigned>(n_seqs)),
+                      dim3(gdn::kChunkThreads), sizeof(gdn::ChunkSmem), s, 1, a);
   // Short sequences stage fewer tokens at a time: a smaller shared-memory footprint,
   // so more CTAs per SM in the state-bound case, and less staging work spent on the
   // empty slots of a chunk (decode: one token per sequence uses the 8-token chunk).
