@@ -305,52 +305,101 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
         }
       }
     }
-    // ---- lower 16 x 16 blocks of K K^T (-> Lt) and Q K^T (-> P split): 20 tasks
-    for (int task = warp; task < 20; task += 8) {
-      const bool is_q = task >= 10;
-      int blk = is_q ? task - 10 : task;  // block (bt, bs), bs <= bt, row-major over the lower triangle
-      int bt = 0;
-      while (blk > bt) {
-        blk -= bt + 1;
-        ++bt;
+    // ---- lower 16 x 16 blocks of K K^T (-> Lt) and Q K^T (-> P split): 20 tasks, warp w
+    // runs tasks w, w + 8, w + 16 side by side (independent accumulators)
+    {
+      constexpr int kTasks = 20, kPer = 3;
+      int bt[kPer], bs[kPer];
+      bool valid[kPer], is_q[kPer];
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) {
+        const int task = warp + 8 * x;
+        valid[x] = task < kTasks;
+        is_q[x] = task >= 10;
+        int blk = valid[x] ? (is_q[x] ? task - 10 : task) : 0;  // row-major over the lower triangle
+        int b = 0;
+        while (blk > b) {
+          blk -= b + 1;
+          ++b;
+        }
+        bt[x] = b;
+        bs[x] = blk;
       }
-      const int bs = blk;
-      float acc[2][4];
+      float acc[kPer][2][4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i)
+      for (int x = 0; x < kPer; ++x)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) acc[i][r] = 0.0f;
-      const uint16_t *A = is_q ? &sm.Q[0][0] : &sm.K[0][0];
-#pragma unroll 4
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) acc[x][i][r] = 0.0f;
+#pragma unroll 2
       for (int kk = 0; kk < kDim / 16; ++kk) {
-        uint32_t af[4], bf[4];
-        ldsm_x4(a_addr(A, kLdKQ, 16 * bt, 16 * kk, lane), af);
-        ldsm_x4(b_addr_nk(&sm.K[0][0], kLdKQ, 16 * bs, 16 * kk, lane), bf);
-        mma16816(acc[0], af, bf[0], bf[1]);
-        mma16816(acc[1], af, bf[2], bf[3]);
+#pragma unroll
+        for (int x = 0; x < kPer; ++x) {
+          if (!valid[x]) continue;  // warp-uniform
+          uint32_t af[4], bf[4];
+          ldsm_x4(a_addr(is_q[x] ? &sm.Q[0][0] : &sm.K[0][0], kLdKQ, 16 * bt[x], 16 * kk, lane), af);
+          ldsm_x4(b_addr_nk(&sm.K[0][0], kLdKQ, 16 * bs[x], 16 * kk, lane), bf);
+          mma16816(acc[x][0], af, bf[0], bf[1]);
+          mma16816(acc[x][1], af, bf[2], bf[3]);
+        }
       }
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int t = 16 * bt + g8 + 8 * hh;
-        const float gt = sm.G[t], gm = t > 0 ? sm.G[t - 1] : 0.0f, be = sm.beta[t];
+      for (int x = 0; x < kPer; ++x) {
+        if (!valid[x]) continue;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int s = 16 * bs + 8 * i + 2 * c4;
-          const float x0 = acc[i][2 * hh], x1 = acc[i][2 * hh + 1];
-          if (is_q) {
-            const float p0 = s <= t ? expf(gt - sm.G[s]) * x0 : 0.0f;
-            const float p1 = s + 1 <= t ? expf(gt - sm.G[s + 1]) * x1 : 0.0f;
-            split2(p0, p1, &sm.Phi[t][s], &sm.Plo[t][s]);
-          } else {
-            sm.Lt[s][t] = s < t ? be * expf(gm - sm.G[s]) * x0 : 0.0f;
-            sm.Lt[s + 1][t] = s + 1 < t ? be * expf(gm - sm.G[s + 1]) * x1 : 0.0f;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int t = 16 * bt[x] + g8 + 8 * hh;
+          const float gt = sm.G[t], gm = t > 0 ? sm.G[t - 1] : 0.0f, be = sm.beta[t];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int s = 16 * bs[x] + 8 * i + 2 * c4;
+            const float x0 = acc[x][i][2 * hh], x1 = acc[x][i][2 * hh + 1];
+            if (is_q[x]) {
+              const float p0 = s <= t ? expf(gt - sm.G[s]) * x0 : 0.0f;
+              const float p1 = s + 1 <= t ? expf(gt - sm.G[s + 1]) * x1 : 0.0f;
+              split2(p0, p1, &sm.Phi[t][s], &sm.Plo[t][s]);
+            } else {
+              sm.Lt[s][t] = s < t ? be * expf(gm - sm.G[s]) * x0 : 0.0f;
+              sm.Lt[s + 1][t] = s + 1 < t ? be * expf(gm - sm.G[s + 1]) * x1 : 0.0f;
+            }
           }
         }
       }
     }
     __syncthreads();
 
-    // ---- (I + L) U = R, right-looking; warp w: columns 8 w .. 8 w + 7
+    // ---- (I + L) U = R, right-looking.  Warp w: columns 8 w .. 8 w + 7; lane (rg, cj):
+    // column 8 w + cj, rows 16 rg .. 16 rg + 15 in registers.  At step t the lane that
+    // holds row t (final by then) broadcasts it with one shuffle and every lane subtracts
+    // L[t'][t] u_t from its rows t'; L[t'][t] = 0 for t' <= t, so finished rows and the
+    // row itself stay as they are.
+    {
+      const int rg = lane >> 3, cj = lane & 7;
+      const int col = 8 * warp + cj;
+      float r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) r[i] = sm.U[16 * rg + i][col];
+#pragma unroll 1
+      for (int tb = 0; tb < kChunk / 16; ++tb) {
+#pragma unroll
+        for (int ti = 0; ti < 16; ++ti) {
+          const float u = __shfl_sync(0xffffffffu, r[ti], tb * 8 + cj);  // row t = 16 tb + ti
+          const float4 *lt = reinterpret_cast<const float4 *>(&sm.Lt[16 * tb + ti][16 * rg]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 l = lt[q];
+            r[4 * q] = fmaf(-l.x, u, r[4 * q]);
+            r[4 * q + 1] = fmaf(-l.y, u, r[4 * q + 1]);
+            r[4 * q + 2] = fmaf(-l.z, u, r[4 * q + 2]);
+            r[4 * q + 3] = fmaf(-l.w, u, r[4 * q + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sm.U[16 * rg + i][col] = r[i];
+    }
+    __syncwarp();  // each warp reads back only its own columns
     {
       const int jw = 8 * warp;
       float r0[8], r1[8];
@@ -361,20 +410,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
         const float4 w = *reinterpret_cast<const float4 *>(&sm.U[lane + 32][jw + 4]);
         r0[0] = p.x, r0[1] = p.y, r0[2] = p.z, r0[3] = p.w, r0[4] = q.x, r0[5] = q.y, r0[6] = q.z, r0[7] = q.w;
         r1[0] = u.x, r1[1] = u.y, r1[2] = u.z, r1[3] = u.w, r1[4] = w.x, r1[5] = w.y, r1[6] = w.z, r1[7] = w.w;
-      }
-#pragma unroll 2
-      for (int t = 0; t < kChunk; ++t) {
-        const int src = t & 31;
-        const bool upper = t >= 32;
-        float u[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) u[e] = __shfl_sync(0xffffffffu, upper ? r1[e] : r0[e], src);
-        const float l0 = sm.Lt[t][lane], l1 = sm.Lt[t][lane + 32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          r0[e] = fmaf(-l0, u[e], r0[e]);
-          r1[e] = fmaf(-l1, u[e], r1[e]);
-        }
       }
       // U and W = diag(e^{G_C - G_s}) U, split for the tensor cores
       const float w0 = sm.wC[lane], w1 = sm.wC[lane + 32];
