@@ -315,7 +315,12 @@ NVFP4_API nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf
  *   update, alpha = forget gate, beta = write strength); alpha = exp(g) follows the log-
  *   space decay the gate epilogue produces (section 機構②).  The read-out S^T q with the
  *   updated state is this library's reading (the pages give none); q and k are used as
- *   given (no normalisation or scaling).  FP32 state and arithmetic.
+ *   given (no normalisation or scaling).  FP32 state.  With 64 or more tokens per
+ *   sequence on average the recurrence runs in its chunked form (64-token chunks, the
+ *   same algebra) with the products on the tensor cores: BF16 q and k, the FP32
+ *   operands split into two BF16 parts, FP32 accumulation, an FP32 triangular solve;
+ *   there g below -80 counts as -80 (a decay below 2e-35).  Otherwise token by token in
+ *   FP32.  Both agree with the exact recurrence within 1e-4 of the output scale.
  *   q, k: device BF16 rows [tokens x ld_qk] (key head hk at column hk*128); v: device
  *   BF16 [tokens x ld_v] (value head h at column h*128); q, k, v 16-byte aligned, ld_qk
  *   and ld_v multiples of 8.  They may be column ranges of one projection output.

@@ -42,7 +42,12 @@ constexpr float kMinLogAlpha = -80.0f;
 constexpr int kLdKQ = kDim + 8;         // BF16 row strides: 8-row ldmatrix groups hit distinct banks
 constexpr int kLdC = kCDV + 8;
 constexpr int kLdT = kChunk + 8;
-constexpr int kLdU = kCDV + 4;          // FP32 rows of R / U (the solve reads rows without conflicts)
+constexpr int kLdU = kCDV + 4;          // FP32 rows of R / U
+constexpr int kLdL = kChunk + 8;        // FP32 rows of L^T, see lt_idx
+
+// L[t][s] is stored at row s (the solve step that reads it), column t, with columns
+// 32 .. 63 shifted by 4: the solve's four row groups then read distinct banks.
+__host__ __device__ constexpr int lt_idx(int s, int t) { return s * kLdL + t + 4 * (t >> 5); }
 
 struct ChunkSmem {
   alignas(16) uint16_t K[kChunk][kLdKQ];    // k_t (BF16), token-major
@@ -57,7 +62,7 @@ struct ChunkSmem {
   alignas(16) uint16_t Whi[kChunk][kLdC];   // W split
   alignas(16) uint16_t Wlo[kChunk][kLdC];
   alignas(16) float U[kChunk][kLdU];        // R, then U after the solve
-  alignas(16) float Lt[kChunk][kChunk];     // Lt[s][t] = L[t][s]
+  alignas(16) float Lt[kChunk * kLdL];      // L[t][s] at lt_idx(s, t)
   float G[kChunk];                          // G_t for t = 1 .. C at index t - 1
   float eG[kChunk];                         // e^{G_t}
   float eGm[kChunk];                        // e^{G_{t-1}}
@@ -65,8 +70,10 @@ struct ChunkSmem {
   float wC[kChunk];                         // e^{G_C - G_s}
 };
 
-// One chunk of inputs in flight in registers: 32 BF16 of k and of q (a quarter of a
-// token's row), 16 BF16 of v, and one token's g and beta.
+// One chunk of inputs in flight in registers.  Rows are read as 16-byte pieces with
+// consecutive lanes on consecutive pieces of a row: piece p = tid + 256 n of k (and q)
+// is token p / 16, d_k columns 8 (p % 16) ..; piece p of v is token p / 8, columns
+// 8 (p % 8) .. of this CTA's block.  Thread t < 64 also holds token t's g and beta.
 struct ChunkStage {
   uint4 k[4], q[4], v[2];
   float g, b;
@@ -76,20 +83,20 @@ __device__ __forceinline__ void chunk_load(const Args &a, ChunkStage &st, int64_
                                            int cb) {
   const int tid = threadIdx.x;
   const uint4 zero = make_uint4(0, 0, 0, 0);
-  {  // k, q: token tid % 64, d_k columns 32 (tid / 64) ..
-    const int64_t tok = t0 + (tid & 63);
-    const int64_t off = tok * a.ld_qk + hk * kDim + (tid >> 6) * 32;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      st.k[n] = tok < end ? __ldg(reinterpret_cast<const uint4 *>(a.k + off) + n) : zero;
-      st.q[n] = tok < end ? __ldg(reinterpret_cast<const uint4 *>(a.q + off) + n) : zero;
-    }
+  for (int n = 0; n < 4; ++n) {
+    const int p = tid + kChunkThreads * n;
+    const int64_t tok = t0 + (p >> 4);
+    const int64_t off = tok * a.ld_qk + hk * kDim + (p & 15) * 8;
+    st.k[n] = tok < end ? __ldg(reinterpret_cast<const uint4 *>(a.k + off)) : zero;
+    st.q[n] = tok < end ? __ldg(reinterpret_cast<const uint4 *>(a.q + off)) : zero;
   }
-  {  // v: token tid / 4, 16 columns from 16 (tid % 4)
-    const int64_t tok = t0 + (tid >> 2);
-    const int64_t off = tok * a.ld_v + h * kDim + cb * kCDV + (tid & 3) * 16;
 #pragma unroll
-    for (int n = 0; n < 2; ++n) st.v[n] = tok < end ? __ldg(reinterpret_cast<const uint4 *>(a.v + off) + n) : zero;
+  for (int n = 0; n < 2; ++n) {
+    const int p = tid + kChunkThreads * n;
+    const int64_t tok = t0 + (p >> 3);
+    const int64_t off = tok * a.ld_v + h * kDim + cb * kCDV + (p & 7) * 8;
+    st.v[n] = tok < end ? __ldg(reinterpret_cast<const uint4 *>(a.v + off)) : zero;
   }
   st.g = 0.0f;
   st.b = 0.0f;
@@ -104,22 +111,53 @@ __device__ __forceinline__ void chunk_load(const Args &a, ChunkStage &st, int64_
 
 __device__ __forceinline__ void chunk_store(ChunkSmem &sm, const ChunkStage &st) {
   const int tid = threadIdx.x;
-  {
-    const int t = tid & 63, i0 = (tid >> 6) * 32;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      *reinterpret_cast<uint4 *>(&sm.K[t][i0 + 8 * n]) = st.k[n];
-      *reinterpret_cast<uint4 *>(&sm.Q[t][i0 + 8 * n]) = st.q[n];
-    }
+  for (int n = 0; n < 4; ++n) {
+    const int p = tid + kChunkThreads * n;
+    *reinterpret_cast<uint4 *>(&sm.K[p >> 4][(p & 15) * 8]) = st.k[n];
+    *reinterpret_cast<uint4 *>(&sm.Q[p >> 4][(p & 15) * 8]) = st.q[n];
   }
-  {
-    const int t = tid >> 2, j0 = (tid & 3) * 16;
 #pragma unroll
-    for (int n = 0; n < 2; ++n) *reinterpret_cast<uint4 *>(&sm.Vb[t][j0 + 8 * n]) = st.v[n];
+  for (int n = 0; n < 2; ++n) {
+    const int p = tid + kChunkThreads * n;
+    *reinterpret_cast<uint4 *>(&sm.Vb[p >> 3][(p & 7) * 8]) = st.v[n];
   }
   if (tid < kChunk) {
     sm.beta[tid] = st.b;
     sm.G[tid] = st.g;  // replaced by the cumulative sums
+  }
+}
+
+// Writes the chunk's outputs, staged as FP32 rows in sm.U, for its first n tokens from
+// token row0: full 16-byte pieces of each row, consecutive lanes on consecutive pieces.
+__device__ __forceinline__ void store_outputs(const Args &a, const ChunkSmem &sm, int64_t row0, int n, int h,
+                                              int cb) {
+  const int tid = threadIdx.x;
+  const int64_t col0 = (int64_t)h * kDim + cb * kCDV;
+  if (a.out_fp32) {  // 16 pieces of 4 floats per row
+#pragma unroll
+    for (int i = 0; i < kChunk * kCDV / 4 / kChunkThreads; ++i) {
+      const int p = tid + kChunkThreads * i;
+      const int t = p >> 4, j = (p & 15) * 4;
+      if (t < n)
+        *reinterpret_cast<float4 *>(static_cast<float *>(a.out) + (row0 + t) * a.ld_out + col0 + j) =
+            *reinterpret_cast<const float4 *>(&sm.U[t][j]);
+    }
+  } else {  // 8 pieces of 8 BF16 per row
+#pragma unroll
+    for (int i = 0; i < kChunk * kCDV / 8 / kChunkThreads; ++i) {
+      const int p = tid + kChunkThreads * i;
+      const int t = p >> 3, j = (p & 7) * 8;
+      if (t < n) {
+        const float4 x = *reinterpret_cast<const float4 *>(&sm.U[t][j]);
+        const float4 y = *reinterpret_cast<const float4 *>(&sm.U[t][j + 4]);
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(x.x, x.y), b1 = __floats2bfloat162_rn(x.z, x.w);
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(y.x, y.y), b3 = __floats2bfloat162_rn(y.z, y.w);
+        *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + (row0 + t) * a.ld_out + col0 + j) =
+            make_uint4(*reinterpret_cast<const uint32_t *>(&b0), *reinterpret_cast<const uint32_t *>(&b1),
+                       *reinterpret_cast<const uint32_t *>(&b2), *reinterpret_cast<const uint32_t *>(&b3));
+      }
+    }
   }
 }
 
@@ -198,7 +236,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
     (&sm.Phi[0][0])[i] = 0;
     (&sm.Plo[0][0])[i] = 0;
   }
-  for (int i = tid; i < kChunk * kChunk; i += kChunkThreads) (&sm.Lt[0][0])[i] = 0.0f;
+  for (int i = tid; i < kChunk * kLdL; i += kChunkThreads) sm.Lt[i] = 0.0f;
   grid_dep_wait();
   grid_dep_launch();
   const int64_t start = __ldg(a.cu_seqlens + b), end = __ldg(a.cu_seqlens + b + 1);
@@ -236,8 +274,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
   const int nh = warp >> 2;  // value columns 32 nh ..
   for (int64_t c = 0; c < nchunks; ++c) {
     const int64_t c0 = start + c * kChunk;
-    const int n = static_cast<int>(end - c0 < kChunk ? end - c0 : kChunk);
     __syncthreads();  // the previous chunk is done with every buffer
+    if (c > 0) store_outputs(a, sm, c0 - kChunk, kChunk, h, cb);  // the previous chunk's (full) outputs
     chunk_store(sm, stg);
     __syncthreads();
     if (warp == 0) {  // G (inclusive prefix), e^G, e^{G_{t-1}}, e^{G_C - G}: tokens lane, lane + 32
@@ -360,8 +398,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
               const float p1 = s + 1 <= t ? expf(gt - sm.G[s + 1]) * x1 : 0.0f;
               split2(p0, p1, &sm.Phi[t][s], &sm.Plo[t][s]);
             } else {
-              sm.Lt[s][t] = s < t ? be * expf(gm - sm.G[s]) * x0 : 0.0f;
-              sm.Lt[s + 1][t] = s + 1 < t ? be * expf(gm - sm.G[s + 1]) * x1 : 0.0f;
+              sm.Lt[lt_idx(s, t)] = s < t ? be * expf(gm - sm.G[s]) * x0 : 0.0f;
+              sm.Lt[lt_idx(s + 1, t)] = s + 1 < t ? be * expf(gm - sm.G[s + 1]) * x1 : 0.0f;
             }
           }
         }
@@ -369,56 +407,60 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
     }
     __syncthreads();
 
-    // ---- (I + L) U = R, right-looking.  Warp w: columns 8 w .. 8 w + 7; lane (rg, cj):
-    // column 8 w + cj, rows 16 rg .. 16 rg + 15 in registers.  At step t the lane that
-    // holds row t (final by then) broadcasts it with one shuffle and every lane subtracts
-    // L[t'][t] u_t from its rows t'; L[t'][t] = 0 for t' <= t, so finished rows and the
-    // row itself stay as they are.
-    {
+    // ---- (I + L) U = R, right-looking, on warps 0 .. 3.  Warp w: columns 16 w .. 16 w + 15;
+    // lane (rg, cj): columns 16 w + 2 cj and + 1, rows 16 rg .. 16 rg + 15 in registers.
+    // At step t the lanes that hold row t (final by then) broadcast it with two shuffles
+    // and every lane subtracts L[t'][t] u_t from its rows t'; L[t'][t] = 0 for t' <= t,
+    // so finished rows and the row itself stay as they are.  U and W =
+    // diag(e^{G_C - G_s}) U are then split for the tensor cores straight from the
+    // registers.  (Eight warps of 8 columns, and two warps holding all 64 rows of a
+    // column each with no shuffles, measured the same or slower.)
+    if (warp < 4) {
       const int rg = lane >> 3, cj = lane & 7;
-      const int col = 8 * warp + cj;
-      float r[16];
+      const int col = 16 * warp + 2 * cj;
+      float r[16][2];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) r[i] = sm.U[16 * rg + i][col];
+      for (int i = 0; i < 16; ++i) {
+        const float2 x = *reinterpret_cast<const float2 *>(&sm.U[16 * rg + i][col]);
+        r[i][0] = x.x;
+        r[i][1] = x.y;
+      }
+      float l[16], ln[16];  // L[16 rg + i][t] for this step and the next
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<float4 *>(&l[4 * q]) = *reinterpret_cast<const float4 *>(&sm.Lt[lt_idx(0, 16 * rg + 4 * q)]);
 #pragma unroll 1
       for (int tb = 0; tb < kChunk / 16; ++tb) {
 #pragma unroll
         for (int ti = 0; ti < 16; ++ti) {
-          const float u = __shfl_sync(0xffffffffu, r[ti], tb * 8 + cj);  // row t = 16 tb + ti
-          const float4 *lt = reinterpret_cast<const float4 *>(&sm.Lt[16 * tb + ti][16 * rg]);
+          const int t = 16 * tb + ti;
+          if (t + 1 < kChunk) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 l = lt[q];
-            r[4 * q] = fmaf(-l.x, u, r[4 * q]);
-            r[4 * q + 1] = fmaf(-l.y, u, r[4 * q + 1]);
-            r[4 * q + 2] = fmaf(-l.z, u, r[4 * q + 2]);
-            r[4 * q + 3] = fmaf(-l.w, u, r[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<float4 *>(&ln[4 * q]) =
+                  *reinterpret_cast<const float4 *>(&sm.Lt[lt_idx(t + 1, 16 * rg + 4 * q)]);
           }
+          const float u0 = __shfl_sync(0xffffffffu, r[ti][0], tb * 8 + cj);  // row t
+          const float u1 = __shfl_sync(0xffffffffu, r[ti][1], tb * 8 + cj);
+          const int nx = (ti + 1) & 15;  // the row the next step broadcasts: update it first
+          r[nx][0] = fmaf(-l[nx], u0, r[nx][0]);
+          r[nx][1] = fmaf(-l[nx], u1, r[nx][1]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i != nx) {
+              r[i][0] = fmaf(-l[i], u0, r[i][0]);
+              r[i][1] = fmaf(-l[i], u1, r[i][1]);
+            }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) l[i] = ln[i];
         }
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) sm.U[16 * rg + i][col] = r[i];
-    }
-    __syncwarp();  // each warp reads back only its own columns
-    {
-      const int jw = 8 * warp;
-      float r0[8], r1[8];
-      {
-        const float4 p = *reinterpret_cast<const float4 *>(&sm.U[lane][jw]);
-        const float4 q = *reinterpret_cast<const float4 *>(&sm.U[lane][jw + 4]);
-        const float4 u = *reinterpret_cast<const float4 *>(&sm.U[lane + 32][jw]);
-        const float4 w = *reinterpret_cast<const float4 *>(&sm.U[lane + 32][jw + 4]);
-        r0[0] = p.x, r0[1] = p.y, r0[2] = p.z, r0[3] = p.w, r0[4] = q.x, r0[5] = q.y, r0[6] = q.z, r0[7] = q.w;
-        r1[0] = u.x, r1[1] = u.y, r1[2] = u.z, r1[3] = u.w, r1[4] = w.x, r1[5] = w.y, r1[6] = w.z, r1[7] = w.w;
-      }
-      // U and W = diag(e^{G_C - G_s}) U, split for the tensor cores
-      const float w0 = sm.wC[lane], w1 = sm.wC[lane + 32];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        split2(r0[e], r0[e + 1], &sm.Uhi[lane][jw + e], &sm.Ulo[lane][jw + e]);
-        split2(r1[e], r1[e + 1], &sm.Uhi[lane + 32][jw + e], &sm.Ulo[lane + 32][jw + e]);
-        split2(w0 * r0[e], w0 * r0[e + 1], &sm.Whi[lane][jw + e], &sm.Wlo[lane][jw + e]);
-        split2(w1 * r1[e], w1 * r1[e + 1], &sm.Whi[lane + 32][jw + e], &sm.Wlo[lane + 32][jw + e]);
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * rg + i;
+        const float w = sm.wC[t];
+        split2(r[i][0], r[i][1], &sm.Uhi[t][col], &sm.Ulo[t][col]);
+        split2(w * r[i][0], w * r[i][1], &sm.Whi[t][col], &sm.Wlo[t][col]);
       }
     }
     __syncthreads();
@@ -448,23 +490,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
           }
         }
       }
+      // staged as FP32 rows in sm.U (no longer needed: U is split) and written out at
+      // the next chunk's first barrier
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int t = 16 * mt + g8 + 8 * hh;
-        if (t >= n) continue;
         const float e = sm.eG[t];
-        const int64_t row = c0 + t;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float y0 = fmaf(e, qs[j][2 * hh], o[j][2 * hh]);
-          const float y1 = fmaf(e, qs[j][2 * hh + 1], o[j][2 * hh + 1]);
-          const int64_t col = (int64_t)h * kDim + cb * kCDV + 32 * nh + 8 * j + 2 * c4;
-          if (a.out_fp32) {
-            *reinterpret_cast<float2 *>(static_cast<float *>(a.out) + row * a.ld_out + col) = make_float2(y0, y1);
-          } else {
-            const __nv_bfloat162 y = __floats2bfloat162_rn(y0, y1);
-            *reinterpret_cast<__nv_bfloat162 *>(static_cast<uint16_t *>(a.out) + row * a.ld_out + col) = y;
-          }
+          const int col = 32 * nh + 8 * j + 2 * c4;
+          *reinterpret_cast<float2 *>(&sm.U[t][col]) =
+              make_float2(fmaf(e, qs[j][2 * hh], o[j][2 * hh]), fmaf(e, qs[j][2 * hh + 1], o[j][2 * hh + 1]));
         }
       }
     }
@@ -493,6 +529,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_kernel(const __grid_co
       }
       write_state_split();  // read by the next chunk after its first two barriers
     }
+  }
+  if (nchunks > 0) {
+    __syncthreads();
+    const int64_t c0 = start + (nchunks - 1) * kChunk;
+    store_outputs(a, sm, c0, static_cast<int>(end - c0), h, cb);
   }
   // final state
 #pragma unroll
