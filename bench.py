@@ -928,7 +928,8 @@ class GDNDecode(GDNRecurrence):
         self.state.copy_(0.3 * torch.randn(self.state.shape, generator=g, device="cuda"))
         self.bytes = M * (32 * 2 * 128 * 128 * 4 + 8192 * 2 + 2 * 32 * 4 + 4096 * 2) + 4.0 * (M + 1)
         self.l2_note = f"states {self.state.numel() * 4 / 1e6:.0f} MB read and written per step (> L2)"
-        self.dominant = ("gdn_recurrence", self.bytes, "hbm", "gdn recurrence_kernel<8> (state read + write)")
+        self.dominant = ("gdn_recurrence", self.bytes, "hbm",
+                         "gdn column_kernel (one warp per four state columns; state read + write)")
         self.phases = {"gdn_recurrence": ("GB/s", self.bytes)}
 
     def work(self):

@@ -321,5 +321,79 @@ __global__ void __launch_bounds__(kThreads) recurrence_kernel(const __grid_const
     }
 }
 
+// ------------------------------------------------------ one warp per state columns
+// Sequences of a few tokens (decode): every state element is read and written once per
+// call, so the pass is HBM-bound, and the column-major state gives each column j of a
+// (sequence, value head) its own contiguous 512 bytes.  One warp owns kColPerWarp
+// columns: lane l holds rows 4 l .. 4 l + 3 of each (one 16-byte load per column, all in
+// flight together), and a token's dot products, S^T k and S^T q per column and k . q,
+// finish with warp reductions:
+//     u = beta (v_j - (S^T k)_j),   S_j <- alpha S_j + u k,   o_j = alpha (S^T q)_j + (k . q) u.
+constexpr int kColWarps = 8;
+constexpr int kColPerWarp = 4;
+constexpr int kColThreads = 32 * kColWarps;
+constexpr int kColBlocksPerHead = kDim / (kColWarps * kColPerWarp);
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Grid (kColBlocksPerHead, H_v, n_seqs), kColThreads threads, no dynamic shared memory.
+__global__ void __launch_bounds__(kColThreads) column_kernel(const __grid_constant__ Args a) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = (blockIdx.x * kColWarps + warp) * kColPerWarp, h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / a.heads_per_key;
+  const int64_t start = __ldg(a.cu_seqlens + b), end = __ldg(a.cu_seqlens + b + 1);
+  if (start < 0 || end < start || end > a.tokens) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicCAS(&g_device_status, 0, kStatusBadIndex);
+    return;
+  }
+  // global [b][h][j][i] holds S[i][j]
+  float4 *col = reinterpret_cast<float4 *>(a.state + (((int64_t)b * gridDim.y + h) * kDim + j0) * kDim) + lane;
+  float4 s[kColPerWarp];
+#pragma unroll
+  for (int c = 0; c < kColPerWarp; ++c) s[c] = a.initial ? col[c * (kDim / 4)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int64_t t = start; t < end; ++t) {
+    const uint2 kw = __ldg(reinterpret_cast<const uint2 *>(a.k + t * a.ld_qk + hk * kDim) + lane);
+    const uint2 qw = __ldg(reinterpret_cast<const uint2 *>(a.q + t * a.ld_qk + hk * kDim) + lane);
+    const float k0 = __uint_as_float(kw.x << 16), k1 = __uint_as_float(kw.x & 0xFFFF0000u);
+    const float k2 = __uint_as_float(kw.y << 16), k3 = __uint_as_float(kw.y & 0xFFFF0000u);
+    const float q0 = __uint_as_float(qw.x << 16), q1 = __uint_as_float(qw.x & 0xFFFF0000u);
+    const float q2 = __uint_as_float(qw.y << 16), q3 = __uint_as_float(qw.y & 0xFFFF0000u);
+    const float alpha = expf(__ldg(a.g + t * a.ld_gate + h));
+    const float be = __ldg(a.beta + t * a.ld_gate + h);
+    const float kq = warp_sum(fmaf(k3, q3, fmaf(k2, q2, fmaf(k1, q1, k0 * q0))));
+#pragma unroll
+    for (int c = 0; c < kColPerWarp; ++c) {
+      const int j = j0 + c;
+      const float vj = __uint_as_float(static_cast<uint32_t>(__ldg(a.v + t * a.ld_v + h * kDim + j)) << 16);
+      float4 &x = s[c];
+      const float sk = warp_sum(fmaf(x.w, k3, fmaf(x.z, k2, fmaf(x.y, k1, x.x * k0))));
+      const float sq = warp_sum(fmaf(x.w, q3, fmaf(x.z, q2, fmaf(x.y, q1, x.x * q0))));
+      const float u = be * (vj - sk);
+      x.x = fmaf(alpha, x.x, k0 * u);
+      x.y = fmaf(alpha, x.y, k1 * u);
+      x.z = fmaf(alpha, x.z, k2 * u);
+      x.w = fmaf(alpha, x.w, k3 * u);
+      if (lane == c) {
+        const float o = fmaf(alpha, sq, kq * u);
+        const int64_t at = t * a.ld_out + (int64_t)h * kDim + j;
+        if (a.out_fp32) {
+          static_cast<float *>(a.out)[at] = o;
+        } else {
+          const __nv_bfloat16 ob = __float2bfloat16_rn(o);
+          static_cast<uint16_t *>(a.out)[at] = *reinterpret_cast<const uint16_t *>(&ob);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kColPerWarp; ++c) col[c * (kDim / 4)] = s[c];
+}
+
 }  // namespace gdn
 }  // namespace nvfp4

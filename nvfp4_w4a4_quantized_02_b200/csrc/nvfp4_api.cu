@@ -663,14 +663,16 @@ nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int6
   if (tokens >= 64 * n_seqs)
     return launch_pdl(gdn::chunk_kernel, dim3(gdn::kChunkColBlocks, n_value_heads, static_cast<unsigned>(n_seqs)),
                       dim3(gdn::kChunkThreads), sizeof(gdn::ChunkSmem), s, 1, a);
-  // Short sequences stage fewer tokens at a time: a smaller shared-memory footprint,
+  // Shorter sequences stage fewer tokens at a time: a smaller shared-memory footprint,
   // so more CTAs per SM in the state-bound case, and less staging work spent on the
-  // empty slots of a chunk (decode: one token per sequence uses the 8-token chunk).
+  // empty slots of a chunk.
   if (tokens >= 16 * n_seqs)
     return launch_pdl(gdn::recurrence_kernel<32>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<32>), s, 1, a);
   if (tokens >= 4 * n_seqs)
     return launch_pdl(gdn::recurrence_kernel<16>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<16>), s, 1, a);
-  return launch_pdl(gdn::recurrence_kernel<8>, grid, dim3(gdn::kThreads), sizeof(gdn::Smem<8>), s, 1, a);
+  // About one token per sequence (decode): one warp per four state columns.
+  return launch_pdl(gdn::column_kernel, dim3(gdn::kColBlocksPerHead, n_value_heads, static_cast<unsigned>(n_seqs)),
+                    dim3(gdn::kColThreads), 0, s, 1, a);
 }
 
 nvfp4_status_t nvfp4_get_device_status(int *code) {

@@ -128,8 +128,8 @@ def test_gdn_long_ragged_sequences(nv, out_dtype, initial):
 
 
 def test_gdn_decode_batch(nv):
-    """Decode: 32 sequences of one token each over a carried state (the short-sequence
-    staging path), all 32 value heads over 16 key heads."""
+    """Decode: 32 sequences of one token each over a carried state (one warp per state
+    column), all 32 value heads over 16 key heads."""
     import torch
     hk, hv, n = 16, 32, 32
     d = synth.gdn_recurrence_inputs([1] * n, hk, hv, seed=152)
@@ -142,6 +142,26 @@ def test_gdn_decode_batch(nv):
     o_ref, s_ref = _oracle(d, hk, hv, S0)
     _check(out.cpu().numpy().reshape(n, hv, 128), o_ref, False)
     _check(state.cpu().numpy().transpose(0, 1, 3, 2), s_ref, False)
+
+
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_gdn_decode_few_tokens(nv, out_dtype):
+    """Under 4 tokens per sequence on average (the one-warp-per-column path): sequences
+    of 3, 1, 0 and 2 tokens, strided rows, a carried state, BF16 and FP32 outputs."""
+    import torch
+    hk, hv = 2, 4
+    lens = [3, 1, 0, 2, 1, 1]
+    d = synth.gdn_recurrence_inputs(lens, hk, hv, seed=159, ld=2 * hk * 128 + hv * 128 + 24)
+    q, k, v, g, b, cu = _dev_inputs(d, hk, hv, gate_ld=hv + 1)
+    rng = np.random.default_rng(160)
+    S0 = (0.3 * rng.standard_normal((len(lens), hv, 128, 128))).astype(np.float32)
+    state = torch.from_numpy(S0).cuda()
+    out = nv.gdn_recurrence(q, k, v, g, b, cu, state, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _oracle(d, hk, hv, S0)
+    _check(out.float().cpu().numpy().reshape(sum(lens), hv, 128), o_ref, out_dtype == "bf16")
+    _check(state.cpu().numpy().transpose(0, 1, 3, 2), s_ref, False)
+    assert nv.device_status() == 0
 
 
 def test_gdn_resuming_from_the_final_state(nv):
@@ -188,20 +208,26 @@ def test_gdn_full_size_sampled_heads(nv):
     assert nv.device_status() == 0
 
 
-def test_gdn_bad_sequence_bounds_are_skipped_and_reported(nv):
+@pytest.mark.parametrize("lens,cu_list", [([1, 2, 1], [0, 1, 0, 4]),         # one warp per column
+                                          ([5, 3], [0, 5, 3, 8]),            # token-by-token kernel
+                                          ([100, 60, 80], [0, 100, 40, 240])])  # chunked kernel
+def test_gdn_bad_sequence_bounds_are_skipped_and_reported(nv, lens, cu_list):
+    """Sequence 1 runs backwards: it is skipped (its state untouched) and reported; the
+    other sequences still run and write their rows."""
     import torch
     hk, hv = 1, 2
-    d = synth.gdn_recurrence_inputs([5, 3], hk, hv, seed=156)
+    T = sum(lens)
+    d = synth.gdn_recurrence_inputs(lens, hk, hv, seed=156)
     q, k, v, g, b, _ = _dev_inputs(d, hk, hv)
-    cu = torch.tensor([0, 5, 3, 8], dtype=torch.int32, device="cuda")  # sequence 1 runs backwards
+    cu = torch.tensor(cu_list, dtype=torch.int32, device="cuda")
     S0 = torch.randn((3, hv, 128, 128), device="cuda")
     state = S0.clone()
-    out = torch.full((8, hv * 128), 7.0, device="cuda")
+    out = torch.full((T, hv * 128), 7.0, device="cuda")
     nv.gdn_recurrence(q, k, v, g, b, cu, state, out=out, out_dtype="f32")
     assert nv.device_status() == 7
     assert torch.equal(state[1], S0[1])
     assert not torch.equal(state[0], S0[0]) and not torch.equal(state[2], S0[2])
-    assert torch.all(out[:5] != 7.0) and torch.all(out[3:8] != 7.0)
+    assert torch.all(out[:cu_list[1]] != 7.0) and torch.all(out[cu_list[2]:T] != 7.0)
 
 
 def test_gdn_strong_decay_and_zero_alpha(nv):
