@@ -4,7 +4,9 @@
 // written to its cache slot as E4M3(fl32(x * fl32(1 / scale))) (nearest even,
 // saturating at +-448, sign kept); a negative slot skips the token.  HBM-bound: 2 bytes
 // read and 1 written per element.  A thread handles one 16-element chunk of a token
-// row in K and the same chunk in V (one slot read for both).
+// row in K and the same chunk in V (one slot read for both); two such chunks are
+// loaded before either is converted, so eight 16-byte loads per thread are in flight
+// (+3 % over one chunk at 32768 and 131072 tokens of width 1024; four chunks were slower).
 #pragma once
 
 #include "quant_math.cuh"
@@ -41,29 +43,44 @@ __global__ void __launch_bounds__(kKvThreads) kv_cache_fp8_kernel(const __grid_c
   grid_dep_wait();
   grid_dep_launch();
   const float k_inv = __frcp_rn(__ldg(a.k_scale)), v_inv = __frcp_rn(__ldg(a.v_scale));
-  const int64_t per_row = a.width / 16;  // 16-element chunks per row
-  // chunk idx = token * per_row + column chunk: shifts when per_row is a power of two
+  const int64_t per_row = a.width / 16;
   const bool pow2 = (per_row & (per_row - 1)) == 0;
   const int shift = __ffsll(per_row) - 1;
   const int64_t total = (int64_t)gridDim.x * kKvThreads;
   const int64_t n = a.tokens * per_row;
-  for (int64_t idx = (int64_t)blockIdx.x * kKvThreads + threadIdx.x; idx < n; idx += total) {
-    const int64_t t = pow2 ? idx >> shift : idx / per_row;
-    const int64_t cc = idx - t * per_row;
-    if (t >= a.tokens) continue;
-    const int64_t slot = __ldg(a.slots + t);
-    if (slot < 0) continue;
-    if (slot >= a.num_slots) {  // never write outside the cache; report it
-      atomicCAS(&g_device_status, 0, kStatusBadIndex);
-      continue;
+  // chunk idx = token * per_row + column chunk: shifts when per_row is a power of two
+  for (int64_t base = (int64_t)blockIdx.x * kKvThreads + threadIdx.x; base < n; base += 2 * total) {
+    uint4 k0[2], k1[2], v0[2], v1[2];  // chunks base and base + total
+    int64_t slot[2], dst[2];           // slot -1: nothing to write
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t idx = base + u * total;
+      slot[u] = -1;
+      if (idx < n) {
+        const int64_t t = pow2 ? idx >> shift : idx / per_row;
+        const int64_t cc = idx - t * per_row;
+        const int64_t sl = __ldg(a.slots + t);
+        if (sl >= a.num_slots) {  // never write outside the cache; report it
+          atomicCAS(&g_device_status, 0, kStatusBadIndex);
+        } else if (sl >= 0) {
+          slot[u] = sl;
+          const int64_t off = t * a.ld + cc * 16;
+          const uint4 *ks = reinterpret_cast<const uint4 *>(a.k + off);
+          const uint4 *vs = reinterpret_cast<const uint4 *>(a.v + off);
+          k0[u] = __ldcs(ks);
+          k1[u] = __ldcs(ks + 1);
+          v0[u] = __ldcs(vs);
+          v1[u] = __ldcs(vs + 1);
+          dst[u] = sl * a.width + cc * 16;
+        }
+      }
     }
-    const int64_t off = t * a.ld + cc * 16;
-    const uint4 *ks = reinterpret_cast<const uint4 *>(a.k + off);
-    const uint4 *vs = reinterpret_cast<const uint4 *>(a.v + off);
-    const uint4 k0 = __ldcs(ks), k1 = __ldcs(ks + 1), v0 = __ldcs(vs), v1 = __ldcs(vs + 1);
-    const int64_t dst = slot * a.width + cc * 16;
-    *reinterpret_cast<uint4 *>(a.k_cache + dst) = fp8_chunk(k0, k1, k_inv);
-    *reinterpret_cast<uint4 *>(a.v_cache + dst) = fp8_chunk(v0, v1, v_inv);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (slot[u] < 0) continue;
+      *reinterpret_cast<uint4 *>(a.k_cache + dst[u]) = fp8_chunk(k0[u], k1[u], k_inv);
+      *reinterpret_cast<uint4 *>(a.v_cache + dst[u]) = fp8_chunk(v0[u], v1[u], v_inv);
+    }
   }
 }
 

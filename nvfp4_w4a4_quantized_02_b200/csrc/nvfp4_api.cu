@@ -615,7 +615,7 @@ nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_
   a.num_slots = num_slots;
   const int64_t chunks = tokens * (width / 16);
   const int64_t want = (chunks + kKvThreads - 1) / kKvThreads;
-  const int64_t cap = int64_t(dev->sms) * 16;
+  const int64_t cap = int64_t(dev->sms) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
   return launch_pdl(kv_cache_fp8_kernel, dim3(grid), dim3(kKvThreads), 0, reinterpret_cast<cudaStream_t>(stream), 1,
                     a);
