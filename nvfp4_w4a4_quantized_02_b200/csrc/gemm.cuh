@@ -791,7 +791,6 @@ constexpr int DEC_W_BYTES = DEC_BM * BK / 2;       // 16 KB
 constexpr int DEC_X_BYTES = DEC_DN_MAX * BK / 2;   // 8 KB
 constexpr int DEC_SF_BYTES = 4 * SF_ATOM;          // 2 KB: 4 k-steps of one 128-row group
 constexpr int DEC_THREADS = 256;                   // producer, MMA, 4 epilogue, 2 copier warps
-constexpr int DEC_EPI_WARP = 2;
 constexpr int DEC_COPY_WARP = 6;
 constexpr uint32_t DEC_ACC_COL = 0;                // DEC_DN_MAX FP32 columns
 constexpr uint32_t DEC_SF_COL = DEC_DN_MAX;        // then one 32-column scale set per stage
