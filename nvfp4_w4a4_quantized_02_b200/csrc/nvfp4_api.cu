@@ -426,8 +426,6 @@ nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t col
     return NVFP4_ERR_MISALIGNED;
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;
-  CUtensorMap tmX;
-  if (!make_bf16_map(&tmX, x_bf16, rows, cols, ld)) return NVFP4_ERR_CUDA;
   QuantArgs a;
   a.gs = gs;
   a.codes = codes;
@@ -441,6 +439,15 @@ nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t col
   a.kb_atoms = (cols + 63) / 64;
   a.tile_r0 = row_offset / 128;
   a.n_tiles = ((a.own_end + 127) / 128 - a.tile_r0) * a.kb_atoms;
+  if (rows <= 64) {  // decode sizes: one thread per 16-element block, no TMA staging
+    const int64_t threads = (a.own_end - row_offset) * 4 * a.kb_atoms;
+    const int64_t blocks = (threads + kQSmallThreads - 1) / kQSmallThreads;
+    if (blocks > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    return launch_pdl(quantize_small_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kQSmallThreads), 0,
+                      reinterpret_cast<cudaStream_t>(stream), 1, static_cast<const uint16_t *>(x_bf16), ld, a);
+  }
+  CUtensorMap tmX;
+  if (!make_bf16_map(&tmX, x_bf16, rows, cols, ld)) return NVFP4_ERR_CUDA;
   const int64_t cap = int64_t(dev->sms) * dev->quant_ctas_per_sm;
   const int grid = static_cast<int>(a.n_tiles < cap ? a.n_tiles : cap);
   return launch_pdl(quantize_kernel, dim3(grid), dim3(kQThreads), kQSmemBytes, reinterpret_cast<cudaStream_t>(stream), 1,

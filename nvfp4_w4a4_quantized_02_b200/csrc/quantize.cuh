@@ -245,4 +245,42 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
   }
 }
 
+// ---------------------------------------------------- a few rows (decode sizes)
+// Up to 64 rows the tile quantiser would stage 128-row tiles that are mostly padding
+// and pay its TMA and barrier set-up for a single tile per CTA.  Here one thread
+// quantises one 16-element block straight from global memory (two 16-byte loads) with
+// quantize16, the same FP32 operations as quantize_kernel, so the output is the same
+// bit for bit.  Scale slots of this call's padding rows and of blocks past `cols` (the
+// 4-block scale words of the last atom column) are written as zero.
+constexpr int kQSmallThreads = 256;
+
+__global__ void __launch_bounds__(kQSmallThreads) quantize_small_kernel(const uint16_t *x, int64_t ld,
+                                                                      const __grid_constant__ QuantArgs a) {
+  grid_dep_wait();  // gs and the input may come from the previous kernel
+  grid_dep_launch();
+  const int64_t slots = 4 * a.kb_atoms;  // scale slots per row
+  const int64_t idx = (int64_t)blockIdx.x * kQSmallThreads + threadIdx.x;
+  if (idx >= (a.own_end - a.row_offset) * slots) return;
+  const int64_t r = idx / slots, kb = idx - r * slots;
+  const int64_t dest = a.row_offset + r;
+  uint8_t *sc = a.scales + scale_word_offset(dest, kb / 4, a.kb_atoms) + (kb & 3);
+  if (r >= a.rows || 16 * kb >= a.cols) {
+    *sc = 0;
+    return;
+  }
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + 16 * kb);
+  const uint4 w0 = __ldg(src), w1 = __ldg(src + 1);
+  const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[2 * j] = __uint_as_float(w[j] << 16);
+    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+  uint32_t c0, c1;
+  const uint32_t sf = quantize16(v, __ldg(a.gs), c0, c1);
+  *reinterpret_cast<uint2 *>(a.codes + dest * a.code_ld + 8 * kb) = make_uint2(c0, c1);
+  *sc = static_cast<uint8_t>(sf);
+}
+
 }  // namespace nvfp4

@@ -58,6 +58,13 @@ def test_ragged_rows_cols_and_leading_dim(nv):
     _check_exact(nv, synth.gaussian_weights(1, 16, seed=5))
 
 
+@pytest.mark.parametrize("rows,cols,ld_pad", [(32, 5120, 0), (64, 4096, 0), (33, 80, 8), (7, 1040, 24)])
+def test_decode_size_rows(nv, rows, cols, ld_pad):
+    """Up to 64 rows (one thread per block, no tile staging): bit-exact codes and scales,
+    padding rows and the blocks past the last column written as zero."""
+    _check_exact(nv, synth.student_t_activations(rows, cols, seed=7 + rows), ld_pad=ld_pad)
+
+
 def test_special_values_pin_rounding_and_sign(nv):
     """Ties, saturation, -0, tiny negatives, zero blocks, exact E2M1 multiples."""
     vals = oracle.e2m1_decode(np.arange(16))
