@@ -990,41 +990,59 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
 }
 
 // ======================================================= split-K epilogue
-// Sums the splits' partials and applies the epilogue of the linear: one thread per
-// 16 output columns of one row (one E4M3 block of an NVFP4 output), so that a
-// decode-size output (tens of rows) still spreads over thousands of threads; rows
-// past M up to the next multiple of 128 only write zero scale bytes (NVFP4 output).
+// Sums the splits' partials and applies the epilogue of the linear, W consecutive
+// output columns of one row per thread: W = 16 (one E4M3 block) for an NVFP4 output,
+// so the thread writes its scale byte itself; W = 4 otherwise, so that a decode-size
+// output (tens of rows) spreads over four times as many threads and loads in flight.
+// Rows past M up to the next multiple of 128 only write zero scale bytes (NVFP4
+// output).  Per output element the splits are added in split order.
 constexpr int REDUCE_THREADS = 256;
 
-// 16 consecutive column sums (col % 16 == 0, col + 16 <= N), added split by split in
-// order, with two splits' loads in flight.
-__device__ __forceinline__ void partial_sum16(const Params &p, int row, int col, float (&y)[16]) {
+// W consecutive column sums (col % W == 0, col + W <= N), added split by split in
+// order, with several splits' loads in flight.
+template <int W>
+__device__ __forceinline__ void partial_sum(const Params &p, int row, int col, float (&y)[W]) {
+  constexpr int V = W / 4;                 // float4 per split
+  constexpr int F = W == 16 ? 2 : 4;       // splits loaded together
 #pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = 0.0f;
-  const int64_t stride = (int64_t)p.M * p.N;
+  for (int i = 0; i < W; ++i) y[i] = 0.0f;
+  const int64_t stride4 = (int64_t)p.M * p.N / 4;
   const float4 *src = reinterpret_cast<const float4 *>(p.partial + (int64_t)row * p.N + col);
   int sp = 0;
-  for (; sp + 2 <= p.splits; sp += 2) {
-    const float4 *s0 = src + sp * (stride / 4), *s1 = src + (sp + 1) * (stride / 4);
-    float4 a[4], b[4];
+  for (; sp + F <= p.splits; sp += F) {
+    float4 a[F][V];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      a[i] = s0[i];
-      b[i] = s1[i];
-    }
+    for (int f = 0; f < F; ++f)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      y[4 * i] += a[i].x, y[4 * i + 1] += a[i].y, y[4 * i + 2] += a[i].z, y[4 * i + 3] += a[i].w;
-      y[4 * i] += b[i].x, y[4 * i + 1] += b[i].y, y[4 * i + 2] += b[i].z, y[4 * i + 3] += b[i].w;
-    }
+      for (int i = 0; i < V; ++i) a[f][i] = src[(sp + f) * stride4 + i];
+#pragma unroll
+    for (int f = 0; f < F; ++f)
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        y[4 * i] += a[f][i].x, y[4 * i + 1] += a[f][i].y, y[4 * i + 2] += a[f][i].z, y[4 * i + 3] += a[f][i].w;
+      }
   }
-  if (sp < p.splits) {
-    const float4 *s0 = src + sp * (stride / 4);
+  for (; sp < p.splits; ++sp) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 a = s0[i];
+    for (int i = 0; i < V; ++i) {
+      const float4 a = src[sp * stride4 + i];
       y[4 * i] += a.x, y[4 * i + 1] += a.y, y[4 * i + 2] += a.z, y[4 * i + 3] += a.w;
     }
+  }
+}
+
+// Store W consecutive BF16 or FP32 outputs of one row.
+template <int W>
+__device__ __forceinline__ void store_w(const Params &p, int row, int col, const float (&y)[W]) {
+  if constexpr (W == 16) {
+    store16(p, row, col, y);
+  } else if (p.out_kind == OUT_BF16) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + col) =
+        make_uint2(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1));
+  } else if (p.out_kind == OUT_F32) {
+    *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (int64_t)row * p.ldo + col) =
+        make_float4(y[0], y[1], y[2], y[3]);
   }
 }
 
@@ -1046,43 +1064,48 @@ __device__ __forceinline__ void store16_nvfp4(const Params &p, const float *inv_
   p.out_scales[scale_word_offset(row, col / 64, p.out_kb_atoms) + (col / 16) % 4] = static_cast<uint8_t>(sf);
 }
 
+template <int W>
 __global__ void __launch_bounds__(REDUCE_THREADS, 1) splitk_epilogue_kernel(const __grid_constant__ Params p) {
   __shared__ Ctrl<1> c;  // segment alphas and the NVFP4 output table
   grid_dep_wait();  // the partial sums come from the previous kernel
   grid_dep_launch();
   load_segments(p, c);
   __syncthreads();
-  const int blocks = p.Nout / 16;  // Nout % 16 == 0
+  const int groups = p.Nout / W;  // Nout % 16 == 0
   const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (int64_t)(p.M + 127) / 128 * 128 : p.M;
   const int64_t idx = (int64_t)blockIdx.x * REDUCE_THREADS + threadIdx.x;
-  if (idx >= rows_cover * blocks) return;
-  const int row = static_cast<int>(idx / blocks);
-  const int col = static_cast<int>(idx - (int64_t)row * blocks) * 16;
-  if (row >= p.M) {
-    p.out_scales[scale_word_offset(row, col / 64, p.out_kb_atoms) + (col / 16) % 4] = 0;
-    return;
+  if (idx >= rows_cover * groups) return;
+  const int row = static_cast<int>(idx / groups);
+  const int col = static_cast<int>(idx - (int64_t)row * groups) * W;
+  if constexpr (W == 16) {
+    if (row >= p.M) {
+      p.out_scales[scale_word_offset(row, col / 64, p.out_kb_atoms) + (col / 16) % 4] = 0;
+      return;
+    }
   }
-  float y[16];
+  float y[W];
   if (p.mode == MODE_SILU_MUL) {
-    float u[16];
-    partial_sum16(p, row, col, y);
-    partial_sum16(p, row, p.up_row0 + col, u);
+    float u[W];
+    partial_sum<W>(p, row, col, y);
+    partial_sum<W>(p, row, p.up_row0 + col, u);
     const float ag = seg_alpha(c, p.nseg, col);
     const float au = seg_alpha(c, p.nseg, p.up_row0 + col);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = silu_mul_f(ag * y[i], au * u[i]);
+    for (int i = 0; i < W; ++i) y[i] = silu_mul_f(ag * y[i], au * u[i]);
   } else {
-    partial_sum16(p, row, col, y);
+    partial_sum<W>(p, row, col, y);
     const float a = seg_alpha(c, p.nseg, col);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] *= a;
+    for (int i = 0; i < W; ++i) y[i] *= a;
   }
-  if (touches_gates(p, col, 16)) gdn_gates<16>(p, row, col, y);
-  if (p.out_kind == OUT_NVFP4) {
-    store16_nvfp4(p, c.inv_out, row, col, y, __ldg(p.gs_out));
-  } else {
-    store16(p, row, col, y);
+  if (touches_gates(p, col, W)) gdn_gates<W>(p, row, col, y);
+  if constexpr (W == 16) {
+    if (p.out_kind == OUT_NVFP4) {
+      store16_nvfp4(p, c.inv_out, row, col, y, __ldg(p.gs_out));
+      return;
+    }
   }
+  store_w<W>(p, row, col, y);
 }
 
 }  // namespace gemm

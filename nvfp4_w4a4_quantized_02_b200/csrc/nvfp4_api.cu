@@ -336,11 +336,14 @@ nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvf
             launch_pdl(gemm_kernel<true>, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p))
       return e;
   }
-  const int64_t rows_cover = p.out_kind == OUT_NVFP4 ? (p.M + 127) / 128 * 128 : p.M;
-  const int64_t threads = rows_cover * (p.Nout / 16);  // one thread per 16-column block
+  // one thread per 16 columns (an E4M3 block) for an NVFP4 output, else per 4 columns
+  const bool nvfp4_out = p.out_kind == OUT_NVFP4;
+  const int64_t rows_cover = nvfp4_out ? (p.M + 127) / 128 * 128 : p.M;
+  const int64_t threads = rows_cover * (p.Nout / (nvfp4_out ? 16 : 4));
   const int64_t blocks = (threads + REDUCE_THREADS - 1) / REDUCE_THREADS;
   if (blocks > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  return launch_pdl(splitk_epilogue_kernel, dim3(static_cast<unsigned>(blocks)), dim3(REDUCE_THREADS), 0, st, 1, p);
+  return launch_pdl(nvfp4_out ? splitk_epilogue_kernel<16> : splitk_epilogue_kernel<4>,
+                    dim3(static_cast<unsigned>(blocks)), dim3(REDUCE_THREADS), 0, st, 1, p);
 }
 
 // ------------------------------------------------- scratch for callers that cannot allocate
