@@ -18,7 +18,7 @@ computes, written from these pages:
   GEMMs.
 
 The pages fix neither a rounding mode, nor an operation order, nor a global-scale
-formula.  The readings taken here (and stated again in the design doc) are:
+formula.  The readings taken here are:
 
 R1  global scale gs = fl32(2688 / amax(|x|)), 2688 = 448 (E4M3 max) * 6 (E2M1 max);
     dequantisation divides by gs; amax == 0 gives gs = 1.
