@@ -539,3 +539,49 @@ def test_gdn_linear_in_values_from_zero_state():
     # value head h reads key head h // 2
     o3, _ = oracle.gdn_recurrence(q[:, :1], k[:, :1], v[:, :2], g[:, :2], b[:, :2])
     assert np.allclose(o3, o1[:, :2], rtol=1e-13)
+
+
+def _chunked_recurrence(q, k, v, g, beta, S0, C):
+    """The recurrence regrouped in chunks of C tokens (the form the prefill kernel
+    evaluates), written out independently of the oracle in FP64.  One value head:
+    q, k [T, d]; v [T, d]; g, beta [T]; S0 [d, d].  Per chunk, with the chunk-local
+    cumulative decays G_t = g_1 + .. + g_t (G_0 = 0):
+        (I + L) U = diag(beta) (V - diag(e^{G_{t-1}}) K S0),
+            L[t, s] = beta_t e^{G_{t-1} - G_s} k_t.k_s  (s < t),
+        O = diag(e^{G_t}) Q S0 + P U,  P[t, s] = e^{G_t - G_s} q_t.k_s  (s <= t),
+        S = e^{G_C} S0 + K^T diag(e^{G_C - G_s}) U."""
+    T = q.shape[0]
+    S = S0.copy()
+    out = np.empty((T, S0.shape[1]))
+    for c0 in range(0, T, C):
+        Q, K, V = q[c0:c0 + C], k[c0:c0 + C], v[c0:c0 + C]
+        n = Q.shape[0]
+        G = np.cumsum(g[c0:c0 + C])
+        Gm = np.concatenate([[0.0], G[:-1]])
+        b = beta[c0:c0 + C]
+        L = np.tril(b[:, None] * np.exp(Gm[:, None] - G[None, :]) * (K @ K.T), -1)
+        R = b[:, None] * (V - np.exp(Gm)[:, None] * (K @ S))
+        U = np.linalg.solve(np.eye(n) + L, R)
+        P = np.tril(np.exp(G[:, None] - G[None, :]) * (Q @ K.T))
+        out[c0:c0 + n] = np.exp(G)[:, None] * (Q @ S) + P @ U
+        S = np.exp(G[-1]) * S + K.T @ (np.exp(G[-1] - G)[:, None] * U)
+    return out, S
+
+
+@pytest.mark.parametrize("T,C", [(150, 64), (64, 64), (7, 4), (33, 16)])
+def test_gdn_chunked_form_equals_the_token_recurrence(T, C):
+    """The chunked regrouping used for long sequences reproduces the token-by-token
+    recurrence (FP64): ragged last chunks, strong and zero decays, a carried state."""
+    rng = np.random.default_rng(143 + T)
+    d = 16
+    q, k = _unit(rng, (T, 1, d)), _unit(rng, (T, 1, d))
+    v = rng.standard_normal((T, 1, d))
+    g = -rng.uniform(0.0, 0.5, (T, 1))
+    g[T // 3] = -30.0    # a near-total forget
+    g[T // 2] = 0.0      # no decay
+    b = rng.uniform(0.05, 1.0, (T, 1))
+    S0 = rng.standard_normal((1, d, d))
+    o_ref, S_ref = oracle.gdn_recurrence(q, k, v, g, b, S0)
+    o, S = _chunked_recurrence(q[:, 0], k[:, 0], v[:, 0], g[:, 0], b[:, 0], S0[0], C)
+    assert np.allclose(o, o_ref[:, 0], rtol=1e-10, atol=1e-10)
+    assert np.allclose(S, S_ref[0], rtol=1e-10, atol=1e-10)
