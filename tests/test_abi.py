@@ -116,3 +116,31 @@ def test_gdn_recurrence_rejects_bad_arguments_without_launch(L):
     assert call(ld_qk=260) == 3                   # row stride not a multiple of 8 BF16
     assert call(state=vp((1 << 20) + 4)) == 3
     assert call(ld_out=516) == 3                  # BF16 out rows must stay 16-byte aligned
+
+
+def test_splitk_rejects_bad_split_and_workspace_without_launch(L):
+    """The split count and the workspace are checked before any device work: split 0 or
+    above K / 256, no workspace, too small or misaligned a workspace; the no-alloc
+    variant rejects partials beyond its fixed scratch array."""
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    A = nv.Operand(1 << 20, 1 << 21, 8, 512)        # 8 rows, K = 512: 2 K tiles
+    W = nv.Operand(1 << 22, 1 << 23, 256, 512)
+    segs = (nv.Segment * 1)(nv.Segment(0, 256, 1 << 24))
+    ep = nv.EpilogueParams()
+    need = L.nvfp4_splitk_workspace_bytes(8, 256, 2)
+
+    def call(split, ws=fake, ws_bytes=need):
+        return L.nvfp4_linear_splitk(ctypes.byref(A), fake, ctypes.byref(W), segs, 1, 0, ctypes.byref(ep), fake, 0,
+                                     256, split, ws, ws_bytes, None)
+    assert call(0) == 1                                 # split 0
+    assert call(3) == 1                                 # more splits than K tiles
+    assert call(2, ws=None) == 1                        # no workspace
+    assert call(2, ws_bytes=need - 16) == 1             # workspace too small
+    assert call(2, ws=vp((1 << 20) + 8)) == 3           # workspace not 16-byte aligned
+    big_W = nv.Operand(1 << 22, 1 << 23, 65536, 512)
+    big_segs = (nv.Segment * 1)(nv.Segment(0, 65536, 1 << 24))
+    big_A = nv.Operand(1 << 20, 1 << 21, 64, 512)
+    # 2 x 64 x 65536 FP32 partials (32 MiB) do not fit the 8 MiB no-alloc scratch
+    assert L.nvfp4_linear_splitk_noalloc(ctypes.byref(big_A), fake, ctypes.byref(big_W), big_segs, 1, 0,
+                                         ctypes.byref(ep), fake, 0, 65536, 2, None) == 2
