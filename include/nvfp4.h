@@ -242,6 +242,10 @@ NVFP4_API int nvfp4_splitk_default(int64_t M, int64_t N, int64_t K);
  *   its contents behind; each call overwrites all of the scratch it reads, so no
  *   state carries over, but calls that overlap on the GPU (other streams, other host
  *   threads) race on it and must be serialised by the caller.
+ *   One split above 64 rows needs no partials: that call runs nvfp4_linear and uses
+ *   no scratch (whatever M * N).  The array's device address is kept per device index
+ *   for the life of the process; a cudaDeviceReset invalidates it, so a process that
+ *   resets a device must not call this entry point on that device again.
  *   Errors: NVFP4_ERR_UNSUPPORTED_SHAPE when split_k * M * N * 4 bytes exceed
  *   NVFP4_NOALLOC_SCRATCH_BYTES (use fewer splits or nvfp4_linear_splitk);
  *   NVFP4_ERR_CUDA if the scratch address cannot be looked up; otherwise as
@@ -253,6 +257,42 @@ NVFP4_API nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, c
                                                      int nseg, int epilogue, const nvfp4_epilogue_params_t *ep,
                                                      void *out, int out_kind, int64_t ldo, int split_k,
                                                      nvfp4_stream_t stream);
+
+/*
+ * nvfp4_unswizzle_scales - the block scales of a packed NVFP4 tensor in logical order.
+ *   out[r * ld + j] = the E4M3 scale byte of row r, 16-element block j, for
+ *   r < rows, j < cols / 16, read from the swizzled buffer `scales` (the layout of the
+ *   conventions above).  For callers that inspect or export scales (checkpoint
+ *   writers, debugging); the GEMM reads the swizzled form directly.
+ *   scales: device, nvfp4_scale_bytes(rows, cols) bytes, 16-byte aligned.
+ *   out: device, rows x ld bytes (any alignment), ld >= cols / 16.  Caller-owned.
+ *   Errors: INVALID_ARG (NULL, rows < 1, ld too small), UNSUPPORTED_SHAPE
+ *   (cols % 16), MISALIGNED (scales).
+ */
+NVFP4_API nvfp4_status_t nvfp4_unswizzle_scales(const uint8_t *scales, int64_t rows, int64_t cols, uint8_t *out,
+                                                int64_t ld, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_pack_weight - pack separately quantised modules into one fused NVFP4 weight
+ * (blog section 罠①: modules fused into one GEMM keep their own global scales; pair
+ * the result with a segment table [(row0_i, row0_i + rows_i, gs_i)] in nvfp4_linear).
+ *   parts[i]: module i, codes [rows_i x K/2] and its own scale buffer (as written by
+ *   nvfp4_quantize), all with the same K.  Module i lands at fused rows
+ *   [row0_i, row0_i + rows_i), row0_i = rows_0 + ... + rows_{i-1} (unaligned offsets
+ *   allowed).  Rows [sum rows_i, rows_out) are padding of the output dimension (for
+ *   example to a multiple of the GEMM's 256-column tile): zero codes, zero scales.
+ *   Scale padding (rows up to a multiple of 128) is written as zero.  The result is
+ *   byte-identical to quantising the modules straight into the fused buffer with
+ *   nvfp4_quantize_rows.  The gate|up order of a SiLU*mul weight needs no interleave:
+ *   the GEMM reads the two halves at their logical offsets.
+ *   codes: device [rows_out x K/2]; scales: device, nvfp4_scale_bytes(rows_out, K)
+ *   bytes; both 16-byte aligned, caller-owned, not overlapping the parts.
+ *   Requirements: 1 <= nparts <= NVFP4_MAX_SEGMENTS, K % 64 == 0, rows_out >= the
+ *   modules' total rows.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE (K % 64),
+ *   MISALIGNED.
+ */
+NVFP4_API nvfp4_status_t nvfp4_pack_weight(const nvfp4_operand_t *parts, int nparts, uint8_t *codes, uint8_t *scales,
+                                           int64_t rows_out, nvfp4_stream_t stream);
 
 /*
  * nvfp4_fold_segments - fused-group scale repair, in place: rewrites a packed fused
@@ -352,6 +392,32 @@ NVFP4_API nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_
  * Synchronises the device.
  */
 NVFP4_API nvfp4_status_t nvfp4_get_device_status(int *code);
+
+/*
+ * nvfp4_selftest_stalled_linear - failure-detection self-test of the bounded waits.
+ * The pages have no counterpart; it checks the library's own guarantee that a kernel
+ * whose pipeline stops never hangs the GPU.  It runs the 1-CTA GEMM of nvfp4_linear
+ * (epilogue NVFP4_EPI_NONE, FP32 output) with one pipeline stage never loaded: the
+ * producer skips stage `stall_stage` (counted from 0 over the K tiles), so the scale
+ * copiers and the MMA issuer wait on a barrier phase that never completes, and the
+ * epilogue waits on an accumulator that is never committed.  In this instantiation
+ * every wait gives up after a short limit (4096 polls instead of the product's
+ * 2^22): each role records NVFP4_ERR_DEVICE_TIMEOUT in the device status word, waits
+ * for the work it already issued, TMEM is freed and the kernel returns.  The output
+ * is left partly written and is meaningless.  The context stays usable: read and
+ * clear the status with nvfp4_get_device_status, after which the other entry points
+ * run as before.
+ *   Arguments as nvfp4_linear with one output tile: A->rows <= 128, W->rows <= 256,
+ *   out FP32 [A->rows x ldo] (device, 16-byte aligned), 0 <= stall_stage < K / 256.
+ *   Errors: NVFP4_ERR_UNSUPPORTED_SHAPE for more than one tile, NVFP4_ERR_INVALID_ARG
+ *   for a stall_stage outside the K tiles, otherwise as nvfp4_linear's checks.
+ *   The call itself returns NVFP4_OK when the launch succeeded; the timeout shows only
+ *   in the status word.
+ */
+NVFP4_API nvfp4_status_t nvfp4_selftest_stalled_linear(const nvfp4_operand_t *A, const float *gs_a,
+                                                       const nvfp4_operand_t *W, const nvfp4_segment_t *segs,
+                                                       int nseg, float *out, int64_t ldo, int stall_stage,
+                                                       nvfp4_stream_t stream);
 
 #ifdef __cplusplus
 }

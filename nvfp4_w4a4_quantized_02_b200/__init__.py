@@ -14,9 +14,9 @@ from typing import Optional, Sequence
 
 __all__ = [
     "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
-    "linear_splitk", "linear_splitk_noalloc", "splitk_default", "splitk_workspace_bytes",
+    "linear_splitk", "linear_splitk_noalloc", "noalloc_default_splits", "splitk_default", "splitk_workspace_bytes",
     "NOALLOC_SCRATCH_BYTES", "fold_segments", "fp8_scale", "kv_cache_fp8", "gdn_recurrence",
-    "device_status", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
+    "device_status", "selftest_stalled_linear", "unswizzle_scales", "pack_weight", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -55,7 +55,8 @@ _LIB = None
 SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_quantize",
            "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
            "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_fold_segments",
-           "nvfp4_fp8_scale", "nvfp4_kv_cache_fp8", "nvfp4_gdn_recurrence", "nvfp4_get_device_status")
+           "nvfp4_fp8_scale", "nvfp4_kv_cache_fp8", "nvfp4_gdn_recurrence", "nvfp4_get_device_status",
+           "nvfp4_selftest_stalled_linear", "nvfp4_unswizzle_scales", "nvfp4_pack_weight")
 
 
 def lib():
@@ -109,6 +110,14 @@ def lib():
                                        _c_vp, _c_i64, ctypes.c_int, _c_vp]
     L.nvfp4_get_device_status.restype = ctypes.c_int
     L.nvfp4_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    L.nvfp4_unswizzle_scales.restype = ctypes.c_int
+    L.nvfp4_unswizzle_scales.argtypes = [_c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp]
+    L.nvfp4_pack_weight.restype = ctypes.c_int
+    L.nvfp4_pack_weight.argtypes = [ctypes.POINTER(Operand), ctypes.c_int, _c_vp, _c_vp, _c_i64, _c_vp]
+    L.nvfp4_selftest_stalled_linear.restype = ctypes.c_int
+    L.nvfp4_selftest_stalled_linear.argtypes = [ctypes.POINTER(Operand), _c_vp, ctypes.POINTER(Operand),
+                                                ctypes.POINTER(Segment), ctypes.c_int, _c_vp, _c_i64, ctypes.c_int,
+                                                _c_vp]
     _LIB = L
     return L
 
@@ -291,6 +300,16 @@ def linear_splitk(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] =
     return result
 
 
+def noalloc_default_splits(M: int, N: int, K: int) -> int:
+    """The library's default split count, lowered until the partial sums fit the fixed
+    scratch array of ``linear_splitk_noalloc`` (never below 1; one split above 64 rows
+    needs no scratch)."""
+    s = max(splitk_default(M, N, K), 1)
+    while s > 1 and splitk_workspace_bytes(M, N, s) > NOALLOC_SCRATCH_BYTES:
+        s -= 1
+    return s
+
+
 def linear_splitk_noalloc(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Sequence] = None,
                           epilogue: str = "none", out_dtype: str = "bf16", out=None, ldo: Optional[int] = None,
                           gates: Optional[dict] = None, gs_out=None, out_scales=None,
@@ -304,10 +323,41 @@ def linear_splitk_noalloc(a: NVFP4Tensor, w: NVFP4Tensor, segments: Optional[Seq
     """
     M, N, K = a.rows, w.rows, a.cols
     if split_k is None:
-        split_k = splitk_default(M, N, K)
+        split_k = noalloc_default_splits(M, N, K)
     args, result, _keep = _linear_args(a, w, segments, epilogue, out_dtype, out, ldo, gates, gs_out, out_scales)
     _check(lib().nvfp4_linear_splitk_noalloc(*args, int(split_k), _stream(stream)), "nvfp4_linear_splitk_noalloc")
     return result
+
+
+def unswizzle_scales(t: NVFP4Tensor, out=None, stream=None):
+    """The E4M3 block scales of ``t`` in logical order: uint8 [rows, cols/16] (device)."""
+    import torch
+    if out is None:
+        out = torch.empty((t.rows, t.cols // 16), dtype=torch.uint8, device=t.scales.device)
+    _check(lib().nvfp4_unswizzle_scales(_c_vp(t.scales.data_ptr()), t.rows, t.cols, _c_vp(out.data_ptr()),
+                                        out.stride(0), _stream(stream)), "nvfp4_unswizzle_scales")
+    return out
+
+
+def pack_weight(parts: Sequence[NVFP4Tensor], rows_out: Optional[int] = None, stream=None):
+    """Pack separately quantised modules (same cols) into one fused NVFP4 weight of
+    ``rows_out`` rows (default: their total; extra rows are zero padding).  Returns
+    ``(NVFP4Tensor, segments)`` with segments ``[(row0, row1, gs), ...]`` of the modules."""
+    import torch
+    cols = parts[0].cols
+    total = sum(p.rows for p in parts)
+    rows_out = total if rows_out is None else rows_out
+    dev = parts[0].codes.device
+    codes = torch.empty((rows_out, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(scale_bytes(rows_out, cols), dtype=torch.uint8, device=dev)
+    ops = (Operand * len(parts))(*[Operand(p.codes.data_ptr(), p.scales.data_ptr(), p.rows, p.cols) for p in parts])
+    _check(lib().nvfp4_pack_weight(ops, len(parts), _c_vp(codes.data_ptr()), _c_vp(scales.data_ptr()), rows_out,
+                                   _stream(stream)), "nvfp4_pack_weight")
+    segs, n0 = [], 0
+    for p in parts:
+        segs.append((n0, n0 + p.rows, p.gs))
+        n0 += p.rows
+    return NVFP4Tensor(codes, scales, parts[0].gs, rows_out, cols), segs
 
 
 def fold_segments(w: NVFP4Tensor, segments: Sequence, gs_out=None, stream=None):
@@ -384,3 +434,18 @@ def device_status() -> int:
     code = ctypes.c_int(0)
     _check(lib().nvfp4_get_device_status(ctypes.byref(code)), "nvfp4_get_device_status")
     return code.value
+
+
+def selftest_stalled_linear(a: NVFP4Tensor, w: NVFP4Tensor, stall_stage: int, stream=None):
+    """Run the failure-detection self-test (``nvfp4_selftest_stalled_linear``): the 1-CTA
+    GEMM with K tile ``stall_stage`` never loaded and short wait limits.  Returns the
+    (meaningless) FP32 output; the timeout shows in ``device_status()``."""
+    import torch
+    out = torch.zeros((a.rows, w.rows), dtype=torch.float32, device=a.codes.device)
+    segs = (Segment * 1)(Segment(0, w.rows, w.gs.data_ptr()))
+    A = Operand(a.codes.data_ptr(), a.scales.data_ptr(), a.rows, a.cols)
+    W = Operand(w.codes.data_ptr(), w.scales.data_ptr(), w.rows, w.cols)
+    _check(lib().nvfp4_selftest_stalled_linear(ctypes.byref(A), _c_vp(a.gs.data_ptr()), ctypes.byref(W), segs, 1,
+                                               _c_vp(out.data_ptr()), out.stride(0), int(stall_stage),
+                                               _stream(stream)), "nvfp4_selftest_stalled_linear")
+    return out

@@ -126,6 +126,9 @@ struct Params {
   int64_t out_kb_atoms;
   // decode kernel: token rows per MMA (32 or 64)
   int dn;
+  // stalled-pipeline self-test only: the producer never loads this stage (counted over
+  // the CTA's run); unused by every product instantiation
+  int stall_stage;
 };
 
 template <int STAGES>
@@ -414,13 +417,13 @@ __device__ __forceinline__ void cp_scale_atom(uint32_t taddr, uint32_t saddr) {
   }
 }
 
-template <int STAGES, bool kPair>
+template <int STAGES, bool kPair, uint32_t kWait = kMaxWaitIters>
 __device__ __forceinline__ void copy_scales(Ctrl<STAGES> &c, uint32_t tmem, const uint8_t *sSFA,
                                             const uint8_t *sSFB, int total, int part) {
   int stage = 0;
   uint32_t phase = 0;
   for (int g = 0; g < total; ++g) {
-    if (!mbar_wait(&c.full[stage], phase)) break;
+    if (!mbar_wait<kWait>(&c.full[stage], phase)) break;
     tc_fence_after();
     const uint32_t sfa = smem_u32(sSFA + stage * SFA_BYTES);
     const uint32_t sfb = smem_u32(sSFB + stage * SFB_BYTES);
@@ -450,7 +453,7 @@ __device__ __forceinline__ void copy_scales(Ctrl<STAGES> &c, uint32_t tmem, cons
   } else {
     tc_commit(drain);
   }
-  mbar_wait(drain, 0);
+  mbar_wait<kWait>(drain, 0);
 }
 
 template <int STAGES>
@@ -472,12 +475,18 @@ __device__ __forceinline__ void init_barriers(Ctrl<STAGES> &c, uint32_t acc_empt
 // epilogue of the linear runs in splitk_epilogue_kernel).  A separate instantiation
 // keeps its code small: a decode-size launch spends much of its few microseconds
 // fetching instructions.
-template <bool kPartial>
+// kStallTest: the failure-detection self-test.  The producer skips stage
+// p.stall_stage (no expected bytes, no loads), so the consumers of that stage wait for
+// a phase that never completes; every wait is capped at kTestWaitIters polls.  Each
+// role then records NVFP4_ERR_DEVICE_TIMEOUT, waits for the work it already issued
+// and leaves; TMEM is freed and the kernel returns.
+template <bool kPartial, bool kStallTest = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ Params p) {
   using P = Plan1;
   constexpr int STAGES = P::STAGES;
+  constexpr uint32_t kWait = kStallTest ? kTestWaitIters : kMaxWaitIters;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl<STAGES> &c = *reinterpret_cast<Ctrl<STAGES> *>(smem);
@@ -513,6 +522,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_phase = 0;  // per-stage bit masks
       bool ok = true;
+      int g = 0;  // stages issued so far (the self-test's stall counter)
       for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
         int tile, split, k0, k1, mt, nt, rb0, rb1;
         unit_coords(p, u, tile, split, k0, k1);
@@ -524,8 +534,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint8_t *sfa_src = p.sfa + ((int64_t)mt * p.kb_atoms) * SF_ATOM;
         const uint8_t *sfb0_src = p.sfb + ((int64_t)(rb0 >> 7) * p.kb_atoms) * SF_ATOM;
         const uint8_t *sfb1_src = p.sfb + ((int64_t)(rb1 >> 7) * p.kb_atoms) * SF_ATOM;
-        for (int kt = k0; kt < k1; ++kt) {
-          if (!mbar_wait(&c.empty[stage], phase ^ 1)) { ok = false; break; }
+        for (int kt = k0; kt < k1; ++kt, ++g) {
+          if (!mbar_wait<kWait>(&c.empty[stage], phase ^ 1)) { ok = false; break; }
+          if constexpr (kStallTest) {
+            if (g == p.stall_stage) {  // never filled: its full barrier stays in this phase
+              if (++stage == STAGES) { stage = 0; phase ^= 1; }
+              continue;
+            }
+          }
           mbar_arrive_expect_tx(&c.full[stage], bytes);
           const int kx = kt * (BK / 2);
           tma_load_2d(sA + stage * A_BYTES, &tmA, &c.full[stage], kx, mt * BM);
@@ -545,7 +561,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // let every copy this thread issued land before the CTA can exit
       for (int s = 0; s < STAGES; ++s)
-        if (armed & (1u << s)) mbar_wait(&c.full[s], (armed_phase >> s) & 1);
+        if (armed & (1u << s)) mbar_wait<kWait>(&c.full[s], (armed_phase >> s) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
@@ -557,11 +573,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
         int tile, split, k0, k1;
         unit_coords(p, u, tile, split, k0, k1);
-        if (!mbar_wait(&c.acc_empty, acc_phase ^ 1)) break;
+        if (!mbar_wait<kWait>(&c.acc_empty, acc_phase ^ 1)) break;
         acc_phase ^= 1;
         tc_fence_after();
         for (int kt = k0; kt < k1; ++kt) {
-          if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
+          if (!mbar_wait<kWait>(&c.full[stage], phase) || !mbar_wait<kWait>(&c.sf_ready[stage], phase)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint64_t a_desc = sdesc_sw128_kmajor(smem_u32(sA + stage * A_BYTES));
           const uint64_t b_desc = sdesc_sw128_kmajor(smem_u32(sB + stage * P::B_BYTES));
@@ -578,7 +597,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // wait for every tcgen05 operation this thread issued
       tc_commit(&c.drain);
-      mbar_wait(&c.drain, 0);
+      mbar_wait<kWait>(&c.drain, 0);
     }
   } else if (warp >= COPY_WARP) {
     if (lane == 0) {
@@ -588,7 +607,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         unit_coords(p, u, tile, split, k0, k1);
         total += k1 - k0;
       }
-      copy_scales<STAGES, false>(c, tmem, sSFA, sSFB, total, warp - COPY_WARP);
+      copy_scales<STAGES, false, kWait>(c, tmem, sSFA, sSFB, total, warp - COPY_WARP);
     }
   } else {
     // ----------------------------------------------------------- epilogue
@@ -607,7 +626,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int tile, split, k0, k1, mt, nt;
       unit_coords(p, u, tile, split, k0, k1);
       tile_coords(p, tile, mt, nt);
-      if (!mbar_wait(&c.acc_full, acc_phase)) break;
+      if (!mbar_wait<kWait>(&c.acc_full, acc_phase)) break;
       acc_phase ^= 1;
       tc_fence_after();
       uint32_t v[4][32];

@@ -4,8 +4,12 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstdint>
+#include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "nvfp4.h"
 #include "quantize.cuh"
@@ -14,6 +18,7 @@
 #include "kvcache.cuh"
 #include "gdn.cuh"
 #include "gdn_chunk.cuh"
+#include "layout.cuh"
 
 using namespace nvfp4;
 
@@ -57,6 +62,8 @@ nvfp4_status_t current_device(DeviceInfo **info) {
                              gemm::Plan1::BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::Plan1::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::gemm_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::Plan1::BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::Plan2::BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -98,6 +105,16 @@ nvfp4_status_t current_device(DeviceInfo **info) {
   return NVFP4_OK;
 }
 
+// NVTX range around one C-ABI call, named after the entry point, so that profilers
+// (Nsight Systems / Compute) show which call launched which kernels.  Without a tool
+// attached each push / pop is a call through a no-op pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -115,10 +132,55 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Cache of encoded tensor maps.  A map is a pure function of (kind, base address,
+// sizes, box), so an entry can never go stale: a buffer freed and reallocated at the
+// same address with the same sizes gets the same map.  Keyed also by device.  The
+// cache is bounded: when full it is cleared and refilled.
+struct MapKey {
+  int dev, kind;
+  const void *ptr;
+  int64_t a, b, c;
+  bool operator==(const MapKey &o) const {
+    return dev == o.dev && kind == o.kind && ptr == o.ptr && a == o.a && b == o.b && c == o.c;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey &k) const {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.ptr) * 0x9E3779B97F4A7C15ull;
+    for (uint64_t v : {uint64_t(k.dev), uint64_t(k.kind), uint64_t(k.a), uint64_t(k.b), uint64_t(k.c)})
+      h = (h ^ v) * 0x100000001B3ull + (h >> 29);
+    return static_cast<size_t>(h);
+  }
+};
+constexpr size_t kMapCacheMax = 4096;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+std::mutex g_maps_mu;
+
+enum MapKind : int { MAP_CODES = 0, MAP_BF16 = 1, MAP_SCALES = 2 };
+
+// Looks `key` up; on a miss runs `encode(m)` and keeps its result.
+template <typename F>
+bool cached_map(CUtensorMap *m, MapKey key, F &&encode) {
+  if (cudaGetDevice(&key.dev) != cudaSuccess) return false;
+  {
+    std::lock_guard<std::mutex> lk(g_maps_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      std::memcpy(m, &it->second, sizeof(CUtensorMap));
+      return true;
+    }
+  }
+  if (!encode(m)) return false;
+  std::lock_guard<std::mutex> lk(g_maps_mu);
+  if (g_maps.size() >= kMapCacheMax) g_maps.clear();
+  g_maps.emplace(key, *m);
+  return true;
+}
+
 // Tensor map of packed codes [rows x K/2] bytes: 128-byte x box_rows boxes with the
 // 128-byte swizzle (the smem layout the MMA descriptors describe); rows beyond
 // `rows` read as zero.
-bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, unsigned box_rows = 128) {
+bool encode_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, unsigned box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
@@ -130,10 +192,15 @@ bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_codes_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, unsigned box_rows = 128) {
+  return cached_map(m, MapKey{0, MAP_CODES, codes, rows, K, box_rows},
+                    [&](CUtensorMap *mm) { return encode_codes_map(mm, codes, rows, K, box_rows); });
+}
+
 // Tensor map of a BF16 matrix [rows x cols] with row stride ld elements: 64-column x
 // 128-row boxes (128 bytes per box row) with the 128-byte swizzle; coordinates
 // outside the matrix read as zero.
-bool make_bf16_map(CUtensorMap *m, const void *x, int64_t rows, int64_t cols, int64_t ld) {
+bool encode_bf16_map(CUtensorMap *m, const void *x, int64_t rows, int64_t cols, int64_t ld) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -145,10 +212,15 @@ bool make_bf16_map(CUtensorMap *m, const void *x, int64_t rows, int64_t cols, in
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_bf16_map(CUtensorMap *m, const void *x, int64_t rows, int64_t cols, int64_t ld) {
+  return cached_map(m, MapKey{0, MAP_BF16, x, rows, cols, ld},
+                    [&](CUtensorMap *mm) { return encode_bf16_map(mm, x, rows, cols, ld); });
+}
+
 // Tensor map of a swizzled scale buffer of a [rows x K] operand, viewed as 8-byte
 // elements: one row per 128-row group (K/64 atoms of 512 bytes), boxes of 256
 // elements = the 4 atoms (2 KB) of one 256-wide K tile of one group.
-bool make_scales_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_t K) {
+bool encode_scales_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_t K) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int64_t groups = (rows + 127) / 128;
@@ -159,6 +231,11 @@ bool make_scales_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_scales_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_t K) {
+  return cached_map(m, MapKey{0, MAP_SCALES, scales, rows, K, 0},
+                    [&](CUtensorMap *mm) { return encode_scales_map(mm, scales, rows, K); });
 }
 
 // Launches `kernel` with programmatic stream serialization: it may begin (shared
@@ -398,6 +475,7 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
 
 nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *gs_out,
                                   nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_global_scale");
   if (!x_bf16 || !gs_out || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
   if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(x_bf16, 16) || ld % 8 != 0 || !aligned(gs_out, 4)) return NVFP4_ERR_MISALIGNED;
@@ -422,6 +500,7 @@ nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols
 nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, const float *gs,
                                    uint8_t *codes, uint8_t *scales, int64_t row_offset, int64_t total_rows,
                                    nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_quantize_rows");
   if (!x_bf16 || !gs || !codes || !scales || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
   if (row_offset < 0 || total_rows < row_offset + rows) return NVFP4_ERR_INVALID_ARG;
   if (cols < 16 || cols % 16 != 0 || total_rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -459,12 +538,14 @@ nvfp4_status_t nvfp4_quantize_rows(const void *x_bf16, int64_t rows, int64_t col
 
 nvfp4_status_t nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, const float *gs,
                               uint8_t *codes, uint8_t *scales, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_quantize");
   return nvfp4_quantize_rows(x_bf16, rows, cols, ld, gs, codes, scales, 0, rows, stream);
 }
 
 nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
                             const nvfp4_segment_t *segs, int nseg, int epilogue, const nvfp4_epilogue_params_t *ep,
                             void *out, int out_kind, int64_t ldo, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_linear");
   using namespace gemm;
   Params p;
   if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, p)) return st;
@@ -508,6 +589,7 @@ nvfp4_status_t nvfp4_linear_splitk(const nvfp4_operand_t *A, const float *gs_a, 
                                    const nvfp4_segment_t *segs, int nseg, int epilogue,
                                    const nvfp4_epilogue_params_t *ep, void *out, int out_kind, int64_t ldo,
                                    int split_k, void *workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_linear_splitk");
   using namespace gemm;
   Params p;
   if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, p)) return st;
@@ -530,10 +612,15 @@ nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, const float
                                            const nvfp4_segment_t *segs, int nseg, int epilogue,
                                            const nvfp4_epilogue_params_t *ep, void *out, int out_kind, int64_t ldo,
                                            int split_k, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_linear_splitk_noalloc");
   using namespace gemm;
   Params p;
   if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, p)) return st;
   if (split_k < 1 || split_k > p.k_tiles) return NVFP4_ERR_INVALID_ARG;
+  // One split above decode size needs no partials: the ordinary kernel, which allocates
+  // nothing either (as in nvfp4_linear_splitk).
+  if (split_k == 1 && p.M > DEC_DN_MAX)
+    return nvfp4_linear(A, gs_a, W, segs, nseg, epilogue, ep, out, out_kind, ldo, stream);
   if (nvfp4_splitk_workspace_bytes(p.M, p.N, split_k) > NVFP4_NOALLOC_SCRATCH_BYTES)
     return NVFP4_ERR_UNSUPPORTED_SHAPE;  // the partials do not fit the fixed scratch array
   DeviceInfo *dev = nullptr;
@@ -543,8 +630,67 @@ nvfp4_status_t nvfp4_linear_splitk_noalloc(const nvfp4_operand_t *A, const float
   return launch_splitk(p, A, W, split_k, scratch, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status_t nvfp4_unswizzle_scales(const uint8_t *scales, int64_t rows, int64_t cols, uint8_t *out, int64_t ld,
+                                      nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_unswizzle_scales");
+  if (!scales || !out || rows < 1 || cols < 16 || ld < cols / 16) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(scales, 16)) return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  UnswizzleArgs a;
+  a.scales = scales;
+  a.out = out;
+  a.rows = rows;
+  a.kb = cols / 16;
+  a.kb_atoms = (a.kb + 3) / 4;
+  a.ld = ld;
+  const int64_t want = (rows * a.kb_atoms + kLayoutThreads - 1) / kLayoutThreads;
+  const int64_t cap = int64_t(dev->sms) * 8;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(unswizzle_scales_kernel, dim3(grid), dim3(kLayoutThreads), 0,
+                    reinterpret_cast<cudaStream_t>(stream), 1, a);
+}
+
+nvfp4_status_t nvfp4_pack_weight(const nvfp4_operand_t *parts, int nparts, uint8_t *codes, uint8_t *scales,
+                                 int64_t rows_out, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_pack_weight");
+  if (!parts || !codes || !scales || nparts < 1 || nparts > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  PackArgs a{};
+  const int64_t K = parts[0].K;
+  int64_t row = 0;
+  for (int i = 0; i < nparts; ++i) {
+    const nvfp4_operand_t &q = parts[i];
+    if (!q.codes || !q.scales || q.rows < 1 || q.K != K) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(q.codes, 16) || !aligned(q.scales, 16)) return NVFP4_ERR_MISALIGNED;
+    a.codes[i] = q.codes;
+    a.scales[i] = q.scales;
+    a.row0[i] = row;
+    row += q.rows;
+  }
+  a.row0[nparts] = row;
+  if (K < 64 || rows_out < row) return NVFP4_ERR_INVALID_ARG;
+  if (K % 64 != 0 || rows_out > kMaxDim || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(codes, 16) || !aligned(scales, 16)) return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  a.nparts = nparts;
+  a.out_codes = codes;
+  a.out_scales = scales;
+  a.rows_out = rows_out;
+  a.code_vecs = K / 32;
+  a.kb_atoms = K / 64;
+  const int64_t tasks = rows_out * a.code_vecs + (rows_out + 127) / 128 * 128 * a.kb_atoms;
+  const int64_t want = (tasks + kLayoutThreads - 1) / kLayoutThreads;
+  const int64_t cap = int64_t(dev->sms) * 8;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(pack_weight_kernel, dim3(grid), dim3(kLayoutThreads), 0, reinterpret_cast<cudaStream_t>(stream), 1,
+                    a);
+}
+
 nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols, const nvfp4_segment_t *segs,
                                    int nseg, float *gs_common_out, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_fold_segments");
   if (!scales || !segs || !gs_common_out || rows < 1 || cols < 1) return NVFP4_ERR_INVALID_ARG;
   if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
   if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -579,6 +725,7 @@ nvfp4_status_t nvfp4_fold_segments(uint8_t *scales, int64_t rows, int64_t cols, 
 
 nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *scale_out,
                                nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_fp8_scale");
   if (!x_bf16 || !scale_out || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
   if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(x_bf16, 16) || ld % 8 != 0 || !aligned(scale_out, 4)) return NVFP4_ERR_MISALIGNED;
@@ -603,6 +750,7 @@ nvfp4_status_t nvfp4_fp8_scale(const void *x_bf16, int64_t rows, int64_t cols, i
 nvfp4_status_t nvfp4_kv_cache_fp8(const void *k_bf16, const void *v_bf16, int64_t tokens, int64_t width,
                                   int64_t ld, const float *k_scale, const float *v_scale, const int64_t *slots,
                                   uint8_t *k_cache, uint8_t *v_cache, int64_t num_slots, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_kv_cache_fp8");
   if (!k_bf16 || !v_bf16 || !k_scale || !v_scale || !slots || !k_cache || !v_cache) return NVFP4_ERR_INVALID_ARG;
   if (tokens < 1 || width < 1 || ld < width || num_slots < 1) return NVFP4_ERR_INVALID_ARG;
   if (width % 16 != 0 || tokens > kMaxDim || width > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -636,6 +784,7 @@ nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int6
                                     const int32_t *cu_seqlens, int64_t n_seqs, int64_t tokens, int n_key_heads,
                                     int n_value_heads, int head_dim, float *state, int initial_state, void *out,
                                     int64_t ld_out, int out_kind, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_gdn_recurrence");
   if (!q_bf16 || !k_bf16 || !v_bf16 || !g || !beta || !cu_seqlens || !state || !out) return NVFP4_ERR_INVALID_ARG;
   if (n_seqs < 1 || tokens < 0 || n_key_heads < 1 || n_value_heads < 1 || n_value_heads % n_key_heads != 0)
     return NVFP4_ERR_INVALID_ARG;
@@ -685,7 +834,29 @@ nvfp4_status_t nvfp4_gdn_recurrence(const void *q_bf16, const void *k_bf16, int6
                     dim3(gdn::kColThreads), 0, s, 1, a);
 }
 
+nvfp4_status_t nvfp4_selftest_stalled_linear(const nvfp4_operand_t *A, const float *gs_a, const nvfp4_operand_t *W,
+                                             const nvfp4_segment_t *segs, int nseg, float *out, int64_t ldo,
+                                             int stall_stage, nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_selftest_stalled_linear");
+  using namespace gemm;
+  Params p;
+  if (nvfp4_status_t st = prepare_linear(A, gs_a, W, segs, nseg, NVFP4_EPI_NONE, nullptr, out, NVFP4_OUT_F32, ldo, p))
+    return st;
+  if (p.M > BM || p.N > BN) return NVFP4_ERR_UNSUPPORTED_SHAPE;  // one tile, one CTA
+  if (stall_stage < 0 || stall_stage >= p.k_tiles) return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  CUtensorMap tmA, tmB;
+  if (!make_codes_map(&tmA, A->codes, p.M, p.K) || !make_codes_map(&tmB, W->codes, p.N, p.K)) return NVFP4_ERR_CUDA;
+  p.m_tiles = 1;
+  p.n_tiles = 1;
+  p.stall_stage = stall_stage;
+  return launch_pdl(gemm_kernel<false, true>, dim3(1), dim3(NUM_THREADS), Plan1::BYTES,
+                    reinterpret_cast<cudaStream_t>(stream), 1, tmA, tmB, p);
+}
+
 nvfp4_status_t nvfp4_get_device_status(int *code) {
+  NvtxRange nvtx("nvfp4_get_device_status");
   if (!code) return NVFP4_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return NVFP4_ERR_CUDA;
   int v = 0, zero = 0;

@@ -15,6 +15,7 @@ __device__ int g_device_status = 0;
 constexpr int kStatusTimeout = 5;          // == NVFP4_ERR_DEVICE_TIMEOUT
 constexpr int kStatusBadIndex = 7;         // == NVFP4_ERR_DEVICE_INDEX
 constexpr uint32_t kMaxWaitIters = 1u << 22;  // try_wait suspends between polls: >= ~0.1 s in total
+constexpr uint32_t kTestWaitIters = 1u << 12;  // the stalled-pipeline self-test's short limit
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -53,10 +54,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with parity `parity` to complete.  Gives up after
-// kMaxWaitIters polls, records a timeout in the status word and returns false.
+// Wait for the phase with parity `parity` to complete.  Gives up after kLimit
+// polls (kMaxWaitIters unless a self-test instantiation asks for fewer), records a
+// timeout in the status word and returns false.
+template <uint32_t kLimit = kMaxWaitIters>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kMaxWaitIters; ++i) {
+  for (uint32_t i = 0; i < kLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
   }
   record_timeout();

@@ -144,3 +144,35 @@ def test_splitk_rejects_bad_split_and_workspace_without_launch(L):
     # 2 x 64 x 65536 FP32 partials (32 MiB) do not fit the 8 MiB no-alloc scratch
     assert L.nvfp4_linear_splitk_noalloc(ctypes.byref(big_A), fake, ctypes.byref(big_W), big_segs, 1, 0,
                                          ctypes.byref(ep), fake, 0, 65536, 2, None) == 2
+
+
+def test_layout_and_selftest_entry_points_reject_bad_arguments_without_launch(L):
+    vp = ctypes.c_void_p
+    f = vp(1 << 20)  # never dereferenced: validation fails first
+    # nvfp4_unswizzle_scales(scales, rows, cols, out, ld, stream)
+    assert L.nvfp4_unswizzle_scales(None, 4, 64, f, 4, None) == 1
+    assert L.nvfp4_unswizzle_scales(f, 0, 64, f, 4, None) == 1
+    assert L.nvfp4_unswizzle_scales(f, 4, 64, f, 3, None) == 1          # ld < cols / 16
+    assert L.nvfp4_unswizzle_scales(f, 4, 72, f, 8, None) == 2          # cols % 16
+    assert L.nvfp4_unswizzle_scales(vp((1 << 20) + 4), 4, 64, f, 4, None) == 3
+    # nvfp4_pack_weight(parts, nparts, codes, scales, rows_out, stream)
+    parts = (nv.Operand * 2)(nv.Operand(1 << 20, 1 << 21, 100, 512), nv.Operand(1 << 22, 1 << 23, 28, 512))
+    assert L.nvfp4_pack_weight(parts, 0, f, f, 128, None) == 1
+    assert L.nvfp4_pack_weight(parts, 2, f, f, 127, None) == 1          # rows_out below the modules' rows
+    assert L.nvfp4_pack_weight(parts, 2, None, f, 128, None) == 1
+    assert L.nvfp4_pack_weight(parts, 2, vp((1 << 20) + 8), f, 128, None) == 3
+    odd = (nv.Operand * 2)(nv.Operand(1 << 20, 1 << 21, 100, 544), nv.Operand(1 << 22, 1 << 23, 28, 544))
+    assert L.nvfp4_pack_weight(odd, 2, f, f, 128, None) == 2            # K % 64
+    mixed = (nv.Operand * 2)(nv.Operand(1 << 20, 1 << 21, 100, 512), nv.Operand(1 << 22, 1 << 23, 28, 1024))
+    assert L.nvfp4_pack_weight(mixed, 2, f, f, 128, None) == 1          # modules of different K
+    # nvfp4_selftest_stalled_linear: one tile only, stall stage inside the K tiles
+    A = nv.Operand(1 << 20, 1 << 21, 128, 512)
+    W = nv.Operand(1 << 22, 1 << 23, 256, 512)
+    segs = (nv.Segment * 1)(nv.Segment(0, 256, 1 << 24))
+    call = lambda A_, W_, s_, stall: L.nvfp4_selftest_stalled_linear(ctypes.byref(A_), f, ctypes.byref(W_), s_, 1,
+                                                                     f, 512, stall, None)
+    assert call(A, W, segs, -1) == 1
+    assert call(A, W, segs, 2) == 1                                       # 2 K tiles
+    W2 = nv.Operand(1 << 22, 1 << 23, 512, 512)
+    segs2 = (nv.Segment * 1)(nv.Segment(0, 512, 1 << 24))
+    assert call(A, W2, segs2, 0) == 2                                     # two output tiles

@@ -85,8 +85,10 @@ def test_mlp_block_full_size_sampled_rows(nv):
     (a) X's global scale and codes (bit-exact);
     (b) gate|up GEMM + SiLU*mul to BF16 against the oracle's FP64 h;
     (c) the fused NVFP4 re-quantisation: bit-equal to the standalone quantiser of (b)'s
-        BF16 output on the whole tensor, and equal to the oracle's codes except where
-        the FP32-vs-FP64 accumulation difference moves h across a rounding midpoint;
+        BF16 output on the whole tensor, bit-equal on the sampled rows to the oracle's
+        quantiser applied to that same BF16 output, and equal to the oracle's codes of
+        its own FP64 h except where the FP32-vs-FP64 accumulation difference moves h
+        across a rounding midpoint;
     (d) the down projection at full size (M = 32768, K = 17408) fed with the oracle's
         own re-quantised rows (zero rows elsewhere), against the oracle."""
     import torch
@@ -132,6 +134,12 @@ def test_mlp_block_full_size_sampled_rows(nv):
     assert torch.equal(hq.codes, hq2.codes) and torch.equal(hq.scales, hq2.scales)
     codes, sf = logical(hq)
     gc, gsf = codes[rows], sf[rows]
+    # bit-exact against the oracle's quantiser applied to the kernel's own BF16 h (the
+    # block format of the next layer's input): every sampled row, codes and scales
+    kc, ks = oracle.quantize(h16[rows_t].float().cpu().numpy(), np.float32(gsh))
+    assert np.array_equal(gc, kc) and np.array_equal(gsf, ks)
+    # end to end against the FP64 h: equal except where the FP32-vs-FP64 accumulation
+    # moves h across a BF16 or E2M1 rounding midpoint
     assert np.mean(gsf == sh) > 0.999
     assert np.mean(gc == ch) > 0.999
     assert rel_fro(oracle.dequantize(gc, gsf, gsh), oracle.dequantize(ch, sh, gsh)) < 1e-2

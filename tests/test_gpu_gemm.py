@@ -181,7 +181,8 @@ def test_gdn_gates_epilogue(nv):
 @pytest.mark.parametrize("M", [256, 300])
 def test_silu_mul_epilogue_and_requant(nv, M):
     """MLP gate|up with SiLU*mul: BF16 output vs oracle, and the fused NVFP4
-    re-quantisation equal (bit for bit) to BF16 output + the standalone quantiser.
+    re-quantisation equal (bit for bit) to BF16 output + the standalone quantiser and
+    to the oracle's quantiser applied to that BF16 output.
     M = 300: the last CTA pair covers rows 256..511, of which 300..383 are scale
     padding (written as zero) and 384..511 lie outside the output."""
     import torch
@@ -210,9 +211,12 @@ def test_silu_mul_epilogue_and_requant(nv, M):
     _sync()
     assert torch.equal(hq.codes, hq2.codes)
     assert torch.equal(hq.scales, hq2.scales)
-    # and against the oracle: codes of h rounded to BF16, quantised with the same gs
-    rc, rsf = oracle.quantize(oracle.round_to_bf16(h_ref).astype(np.float32), np.float32(gs_h.item()))
     gc, gsf = logical(hq)
+    # bit-exact against the oracle's quantiser applied to the kernel's own BF16 h
+    kc, ks = oracle.quantize(h16.float().cpu().numpy(), np.float32(gs_h.item()))
+    assert np.array_equal(gc, kc) and np.array_equal(gsf, ks)
+    # and end to end: codes of the oracle's FP64 h rounded to BF16, with the same gs
+    rc, rsf = oracle.quantize(oracle.round_to_bf16(h_ref).astype(np.float32), np.float32(gs_h.item()))
     assert np.mean(gsf == rsf) > 0.995
     assert np.mean(gc == rc) > 0.995
     deq_g = oracle.dequantize(gc, gsf, gs_h.item())

@@ -123,7 +123,8 @@ def test_gdn_inproj_decode_full_size(nv, split_k):
 @pytest.mark.parametrize("split_k", [1, 3, 4])
 def test_silu_mul_requant_decode(nv, split_k):
     """Gate|up with SiLU*mul and NVFP4 re-quantisation: BF16 output against the oracle;
-    the NVFP4 output equals the standalone quantiser applied to the BF16 output.  With
+    the NVFP4 output equals the standalone quantiser applied to the BF16 output, and
+    the oracle's quantiser applied to it.  With
     4 K tiles, splits 1, 3 (two K ranges of 2, so 2 splits) and 4."""
     import torch
     M, K, Nh = 32, 1024, 2048
@@ -149,8 +150,11 @@ def test_silu_mul_requant_decode(nv, split_k):
     hq2 = nv.quantize(h16, gs_h)
     _sync()
     assert torch.equal(hq.codes, hq2.codes) and torch.equal(hq.scales, hq2.scales)
-    rc, rsf = oracle.quantize(oracle.round_to_bf16(h_ref).astype(np.float32), np.float32(gs_h.item()))
     gc, gsf = logical(hq)
+    # bit-exact against the oracle's quantiser applied to the kernel's own BF16 h
+    kc, ks = oracle.quantize(h16.float().cpu().numpy(), np.float32(gs_h.item()))
+    assert np.array_equal(gc, kc) and np.array_equal(gsf, ks)
+    rc, rsf = oracle.quantize(oracle.round_to_bf16(h_ref).astype(np.float32), np.float32(gs_h.item()))
     assert np.mean(gc == rc) > 0.995 and np.mean(gsf == rsf) > 0.995
 
 
