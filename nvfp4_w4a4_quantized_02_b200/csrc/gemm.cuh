@@ -24,7 +24,11 @@
 //   warp 0      TMA producer: code tiles (128-byte swizzle) and scale tiles (already
 //               in the MMA's 128 x 4 atom layout) into a shared-memory ring.
 //   warp 1      MMA issuer: 4 block-scaled MMAs (K = 64 each) per stage into the
-//               TMEM accumulator, then frees the stage with tcgen05.commit.
+//               TMEM accumulator, then frees the stage with tcgen05.commit.  It waits on
+//               one barrier per stage, sf_ready: the copiers copy a stage's scales only
+//               after its bytes landed, so their commit covers the operands too.  (A
+//               second wait on the stage's load barrier cost ~190 cycles of the issuer's
+//               per-stage loop: 2.47 -> 2.27 ms on the MLP block's gate|up GEMM.)
 //   warps 2..9  epilogue: tcgen05.ld the 128 x 256 FP32 accumulator (each warp a
 //               32-lane quadrant x 128 columns) into registers, hand TMEM back to the
 //               MMA warp at once, then scale / activate / store from registers.
@@ -577,10 +581,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1;
         tc_fence_after();
         for (int kt = k0; kt < k1; ++kt) {
-          if (!mbar_wait<kWait>(&c.full[stage], phase) || !mbar_wait<kWait>(&c.sf_ready[stage], phase)) {
-            ok = false;
-            break;
-          }
+          // sf_ready completes only after a copier saw full[stage] (the stage's bytes
+          // landed) and its copies of the stage's scales completed: one wait covers both.
+          if (!mbar_wait<kWait>(&c.sf_ready[stage], phase)) { ok = false; break; }
           tc_fence_after();
           const uint64_t a_desc = sdesc_sw128_kmajor(smem_u32(sA + stage * A_BYTES));
           const uint64_t b_desc = sdesc_sw128_kmajor(smem_u32(sB + stage * P::B_BYTES));
@@ -740,7 +743,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1;
         tc_fence_after();
         for (int kt = 0; kt < p.k_tiles; ++kt) {
-          if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
+          if (!mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }  // implies full[stage]
           tc_fence_after();
           const uint64_t a_desc = sdesc_sw128_kmajor(smem_u32(sA + stage * A_BYTES));
           const uint64_t b_desc = sdesc_sw128_kmajor(smem_u32(sB + stage * P::B_BYTES));
@@ -925,7 +928,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
         acc_phase ^= 1;
         tc_fence_after();
         for (int kt = k0; kt < k1; ++kt) {
-          if (!mbar_wait(&c.full[stage], phase) || !mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }
+          if (!mbar_wait(&c.sf_ready[stage], phase)) { ok = false; break; }  // implies full[stage]
           tc_fence_after();
           const uint64_t w_desc = sdesc_sw128_kmajor(smem_u32(sW + stage * DEC_W_BYTES));
           const uint64_t x_desc = sdesc_sw128_kmajor(smem_u32(sX + stage * DEC_X_BYTES));
