@@ -877,12 +877,18 @@ class GDNRecurrence(Workload):
         self.state = torch.zeros((self.n_seqs, 32, 128, 128), dtype=torch.float32, device="cuda")
         self.out = torch.empty((M, 32 * 128), dtype=torch.bfloat16, device="cuda")
         self.flops = 7.0 * 128 * 128 * 32 * M
+        # Tensor-core FLOPs chunk_kernel issues: per (64-token chunk, value head, 64-column
+        # block) 2096 mma.sync m16n8k16 (K S0 / Q S0 hi+lo 1024, lower K K^T / Q K^T blocks
+        # 320, P U as three split products over the lower triangle 240, K^T W hi+lo 512),
+        # 4096 FLOP each; two column blocks per head.
+        chunks = sum(-(-min(self.SEQ, M - s0) // 64) for s0 in range(0, M, self.SEQ))
+        self.mma_flops = 2096.0 * 4096 * chunks * 32 * 2
         self.launches_per_step = 1
         self.l2_note = (f"inputs larger than L2 (q|k|v rows {M * 8192 * 2 / 1e6:.0f} MB, out "
                         f"{M * 4096 * 2 / 1e6:.0f} MB)")
-        self.dominant = ("gdn_recurrence", self.flops, "alu",
+        self.dominant = ("gdn_recurrence", self.mma_flops, "tensor_bf16",
                          "gdn chunk_kernel (64-token chunks; products on BF16 mma.sync with FP32 operands split "
-                         "hi/lo; rate in the token recurrence's FLOPs)")
+                         "hi/lo; rate in the tensor FLOPs it issues, against the BF16 tensor peak)")
         self.phases = {"gdn_recurrence": ("ALU", self.flops)}
         torch.cuda.synchronize()
 
@@ -892,7 +898,8 @@ class GDNRecurrence(Workload):
     def config(self):
         return {"tokens": self.M, "seq_len": min(self.M, self.SEQ), "n_seqs": self.n_seqs, "key_heads": 16,
                 "value_heads": 32, "head_dim": 128, "state": "fp32, fresh per sequence",
-                "flops_per_token_head": "7 * 128 * 128"}
+                "flops_per_token_head": "7 * 128 * 128 (token recurrence)",
+                "tensor_flops_issued_per_launch": self.mma_flops}
 
     def plan(self, x):
         nv = self.nv
@@ -1119,6 +1126,14 @@ def run_ours(args, ws, rank):
         peak, unit = round(alu_peak, 2), "TFLOP/s"
         note = (f"derived FP32 FMA peak: {props.multi_processor_count} SMs x {FP32_LANES_PER_SM} lanes x 2 FLOP x "
                 f"{sm_max:.0f} MHz")
+    elif bound == "tensor_bf16":
+        achieved = per_launch / avg_ms / 1e9
+        peak, unit = round(bf16_peak, 1), "TFLOP/s"
+        bound = "tensor"
+        src = "bf16_tflops_sustained" if region == "sustained" else "bf16_tflops (burst)"
+        note = f"{peak_src} {src} (BF16 mma.sync products); timed region {elapsed_ms:.0f} ms"
+        extra_fracs = {"frac_nominal": round(achieved / (NOMINAL_FP4_TFLOPS / FP4_OVER_BF16), 4),
+                       "nominal_peak": NOMINAL_FP4_TFLOPS / FP4_OVER_BF16}
     else:
         achieved = per_launch / avg_ms / 1e9
         peak, unit = round(fp4_peak, 1), "TFLOP/s"

@@ -167,6 +167,15 @@ __device__ __forceinline__ void tile_coords(const Params &p, int tile, int &mt, 
   nt = idx / gm;
 }
 
+// MMA N of N-tile nt: BN, or for a narrower last tile its valid width rounded up to 32
+// (the CTA pair then holds half of it per CTA, a multiple of 16 rows), so that the tail
+// tile of, e.g., a 12352-row fused weight runs a quarter-width MMA instead of a full one.
+// SILU_MUL tiles are always full (N % 256 == 0).
+__device__ __forceinline__ int tile_mma_n(const Params &p, int nt) {
+  const int w = p.N - nt * BN;
+  return (p.tile_mode == MODE_SILU_MUL || w >= BN) ? BN : (w + 31) / 32 * 32;
+}
+
 // First weight rows of the two 128-row halves of the B tile of N-tile nt.
 __device__ __forceinline__ void b_rows(const Params &p, int nt, int &rb0, int &rb1) {
   if (p.tile_mode == MODE_SILU_MUL) {
@@ -570,13 +579,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(BM, BN);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-        int tile, split, k0, k1;
+        int tile, split, k0, k1, mt, nt;
         unit_coords(p, u, tile, split, k0, k1);
+        tile_coords(p, tile, mt, nt);
+        const uint32_t idesc = make_idesc(BM, tile_mma_n(p, nt));  // B rows 0.. of the tile
         if (!mbar_wait<kWait>(&c.acc_empty, acc_phase ^ 1)) break;
         acc_phase ^= 1;
         tc_fence_after();
@@ -709,7 +719,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_coords(p, tile, mt, nt);
         b_rows(p, nt, rb0, rb1);
         const int a_row = mt * (2 * BM) + (int)rank * BM;
-        const int b_row = rank == 0 ? rb0 : rb1;
+        const int n_mma = tile_mma_n(p, nt);  // the CTA pair splits the MMA's N rows of B in halves
+        const int b_row = rank == 0 ? rb0 : (n_mma == BN ? rb1 : rb0 + n_mma / 2);
         for (int kt = 0; kt < p.k_tiles; ++kt) {
           if (!mbar_wait(&c.empty[stage], phase ^ 1)) { ok = false; break; }
           if (rank == 0) mbar_arrive_expect_tx(&c.full[stage], 2 * STAGE2_TX);
@@ -734,11 +745,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = make_idesc(2 * BM, BN);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
+        int mt, nt;
+        tile_coords(p, tile, mt, nt);
+        const uint32_t idesc = make_idesc(2 * BM, tile_mma_n(p, nt));
         if (!mbar_wait_cluster(&c.acc_empty, acc_phase ^ 1)) break;
         acc_phase ^= 1;
         tc_fence_after();

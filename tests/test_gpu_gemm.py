@@ -60,6 +60,25 @@ def test_exact_power_of_two_scales_pin_scale_layout(nv):
     assert np.array_equal(got, ref), f"{np.sum(got != ref)} mismatches"
 
 
+@pytest.mark.parametrize("M,N", [(100, 80), (256, 16), (256, 48), (256, 336), (300, 464), (512, 272), (128, 208)])
+def test_exact_narrow_last_n_tile(nv, M, N):
+    """The last N-tile narrower than 256 runs an MMA of N = its width rounded up to 32;
+    in the CTA pair the second CTA then holds B rows [N/2, N) of the tile.  Integer codes
+    and unit scales keep the FP32 result exact, so any misplaced B row shows."""
+    rng = np.random.default_rng(M * 1000 + N)
+    K = 512
+    ca = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    cw = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sa = np.full((M, K // 16), 0x38, np.uint8)
+    sw = np.full((N, K // 16), 0x38, np.uint8)
+    ref = oracle.linear(ca, sa, 1.0, cw, sw, [(0, N, 1.0)])
+    out = nv.linear(make_operand(ca, sa, 1.0), make_operand(cw, sw, 1.0), out_dtype="f32")
+    _sync()
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got, ref), f"{np.sum(got != ref)} mismatches"
+    assert nv.device_status() == 0
+
+
 @pytest.mark.parametrize("M", [128, 256])
 def test_single_nonzero_probes(nv, M):
     """One non-zero code / scale at a time lands in exactly one output element.
