@@ -1293,7 +1293,9 @@ def run_e2e(wl, args, torch, flush, g_step=None):
     return {"value": round(wl.work() / (ms * 1e-3) / scale, 2), "unit": wl.unit,
             "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
             "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
-            "ms_per_step": round(ms, 4), "steps": n, "schedule": "sequential, L2 flushed between steps"}
+            "ms_per_step": round(ms, 4), "steps": n, "schedule": "sequential, L2 flushed between steps",
+            "host_leg": "pinned host buffers and torch copies around the Python binding's C-ABI calls (the C ABI "
+                        "itself takes device pointers)"}
 
 
 def run_e2e_pipelined(wl, args, torch, g_step=None):
@@ -1352,7 +1354,9 @@ def run_e2e_pipelined(wl, args, torch, g_step=None):
             "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(),
             "ms_per_step": round(ms, 4), "steps": n,
             "schedule": "pipelined: H2D of step i+1 and D2H of step i-1 overlap step i (two copy streams, "
-                        "double-buffered device staging)"}
+                        "double-buffered device staging)",
+            "host_leg": "pinned host buffers and torch copies around the Python binding's C-ABI calls (the C ABI "
+                        "itself takes device pointers)"}
 
 
 # ---------------------------------------------------------------- CPU oracle

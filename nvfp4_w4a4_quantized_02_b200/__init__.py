@@ -20,7 +20,10 @@ __all__ = [
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libnvfp4_w4a4.so")
+# NVFP4_DEBUG=1 selects the bounds-checking build of the same library (built with
+# ``python -m nvfp4_w4a4_quantized_02_b200.build --debug``).
+DEBUG = os.environ.get("NVFP4_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libnvfp4_w4a4_debug.so" if DEBUG else "libnvfp4_w4a4.so")
 
 EPILOGUES = {"none": 0, "silu_mul": 1, "gdn_gates": 2}
 OUT_KINDS = {"bf16": 0, "f32": 1, "nvfp4": 2}
@@ -67,7 +70,7 @@ def lib():
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
             f"NVFP4 CUDA library not built ({LIB_PATH} missing): "
-            "run `python -m nvfp4_w4a4_quantized_02_b200.build`")
+            f"run `python -m nvfp4_w4a4_quantized_02_b200.build{' --debug' if DEBUG else ''}`")
     L = ctypes.CDLL(LIB_PATH)
     L.nvfp4_status_string.restype = ctypes.c_char_p
     L.nvfp4_status_string.argtypes = [ctypes.c_int]

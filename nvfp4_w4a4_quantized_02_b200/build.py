@@ -18,6 +18,11 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libnvfp4_w4a4.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
+# The bounds-checking build: the same sources with -DNVFP4_DEBUG, in which every global
+# store of the GEMM and quantiser kernels first checks its index invariants, records
+# NVFP4_ERR_DEVICE_INDEX and skips the store when one fails.  Loaded by the Python
+# binding when the environment sets NVFP4_DEBUG=1.
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libnvfp4_w4a4_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -39,19 +44,22 @@ def _sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB_PATH):
+def needs_build(debug: bool = False) -> bool:
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if it is missing or older than its sources; return its path."""
-    if not force and not needs_build():
-        return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC,
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile the library (``debug``: the bounds-checking build) if it is missing or
+    older than its sources; return its path."""
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not force and not needs_build(debug):
+        return path
+    tmp = path + ".tmp"
+    cmd = [_nvcc(), *NVCC_FLAGS, *(["-DNVFP4_DEBUG"] if debug else []), "-I", INCLUDE, "-I", CSRC,
            "-o", tmp, os.path.join(CSRC, "nvfp4_api.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -61,9 +69,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         print(res.stdout + res.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -133,6 +133,8 @@ struct Params {
   // stalled-pipeline self-test only: the producer never loads this stage (counted over
   // the CTA's run); unused by every product instantiation
   int stall_stage;
+  // the output's base and row stride are 32-byte aligned: stores of 32 bytes per lane
+  int st32;
 };
 
 template <int STAGES>
@@ -203,6 +205,23 @@ __device__ __forceinline__ float seg_alpha(const Ctrl<STAGES> &c, int nseg, int 
   return a;
 }
 
+// Alphas of the four 16-column blocks [n0, n0 + 64): one lookup when the group lies in
+// one segment (segments are sorted, contiguous from column 0 and 16-aligned), else one
+// per block.  The epilogue's instruction count matters: its warps share the issue slots
+// of the producer, copier and MMA threads.
+template <int STAGES>
+__device__ __forceinline__ void seg_alpha4(const Ctrl<STAGES> &c, int nseg, int n0, float (&a)[4]) {
+  int s = 0;
+  while (s + 1 < nseg && n0 >= c.seg_end[s]) ++s;
+  if (n0 >= c.seg_begin[s] && n0 + 64 <= c.seg_end[s]) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) a[b] = c.seg_alpha[s];
+  } else {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) a[b] = seg_alpha(c, nseg, n0 + 16 * b);
+  }
+}
+
 // Gate and activation functions with the hardware approximations (relative error of
 // order 1e-6: far below the BF16 store and the 1e-3 bar of the gates).  softplus uses
 // the stable form max(x, 0) + log(1 + e^-|x|); 1 + e^-|x| lies in (1, 2], where the
@@ -213,6 +232,7 @@ __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.0f) + _
 
 // Store 16 consecutive output values of one row.
 __device__ __forceinline__ void store16(const Params &p, int row, int col, const float (&y)[16]) {
+  if (!NVFP4_DCHECK(row >= 0 && row < p.M && col >= 0 && col % 16 == 0 && col + 16 <= p.Nout)) return;
   if (p.out_kind == OUT_BF16) {
     uint32_t w[8];
 #pragma unroll
@@ -220,13 +240,29 @@ __device__ __forceinline__ void store16(const Params &p, int row, int col, const
       __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
       w[i] = *reinterpret_cast<uint32_t *>(&h);
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + col);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    __nv_bfloat16 *d = static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + col;
+    if (p.st32) {
+      st_global_v8(d, w);
+    } else {
+      uint4 *dst = reinterpret_cast<uint4 *>(d);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
   } else if (p.out_kind == OUT_F32) {
-    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (int64_t)row * p.ldo + col);
+    float *d = static_cast<float *>(p.out) + (int64_t)row * p.ldo + col;
+    if (p.st32) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(y[8 * h + i]);
+        st_global_v8(d + 8 * h, w);
+      }
+    } else {
+      float4 *dst = reinterpret_cast<float4 *>(d);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+    }
   }
 }
 
@@ -235,6 +271,7 @@ __device__ __forceinline__ void store16(const Params &p, int row, int col, const
 // read from the CTA's table, the same FP32 division).
 __device__ __forceinline__ void store64_nvfp4(const Params &p, const float *inv_out, int row, int col,
                                               const float (&y)[64], float gs_out) {
+  if (!NVFP4_DCHECK(row >= 0 && row < p.M && col >= 0 && col % 64 == 0 && col + 64 <= p.Nout)) return;
   uint32_t codes[8];
   uint32_t sfword = 0;
 #pragma unroll
@@ -252,9 +289,14 @@ __device__ __forceinline__ void store64_nvfp4(const Params &p, const float *inv_
     codes[2 * b + 1] = encode8(x + 8, inv);
     sfword |= sf << (8 * b);
   }
-  uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) + (int64_t)row * (p.Nout / 2) + col / 2);
-  dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-  dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+  uint8_t *d = static_cast<uint8_t *>(p.out) + (int64_t)row * (p.Nout / 2) + col / 2;
+  if (p.st32) {
+    st_global_v8(d, codes);
+  } else {
+    uint4 *dst = reinterpret_cast<uint4 *>(d);
+    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+  }
   *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, col / 64, p.out_kb_atoms)) = sfword;
 }
 
@@ -269,11 +311,12 @@ __device__ __forceinline__ void gdn_gates(const Params &p, int row, int cg, floa
     const int n = cg + i;
     if (n >= p.beta_begin && n < p.beta_begin + p.n_heads) {
       y[i] = sigmoid_f(y[i]);
-      if (p.beta_out) p.beta_out[(int64_t)row * p.n_heads + (n - p.beta_begin)] = y[i];
+      if (p.beta_out && NVFP4_DCHECK(row >= 0 && row < p.M))
+        p.beta_out[(int64_t)row * p.n_heads + (n - p.beta_begin)] = y[i];
     } else if (n >= p.alpha_begin && n < p.alpha_begin + p.n_heads) {
       const int hh = n - p.alpha_begin;
       y[i] = -__expf(__ldg(p.A_log + hh)) * softplus_f(y[i] + __ldg(p.dt_bias + hh));
-      if (p.g_out) p.g_out[(int64_t)row * p.n_heads + hh] = y[i];
+      if (p.g_out && NVFP4_DCHECK(row >= 0 && row < p.M)) p.g_out[(int64_t)row * p.n_heads + hh] = y[i];
     }
   }
 }
@@ -314,7 +357,8 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
       const int rows_pad = (p.M + 127) / 128 * 128;
       if (row < rows_pad)
         for (int cg = cbeg; cg < cbeg + span && cg < p.Nout; cg += 64)
-          *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, cg / 64, p.out_kb_atoms)) = 0u;
+          if (NVFP4_DCHECK(cg % 64 == 0 && cg / 64 < p.out_kb_atoms))
+            *reinterpret_cast<uint32_t *>(p.out_scales + scale_word_offset(row, cg / 64, p.out_kb_atoms)) = 0u;
     }
     return;
   }
@@ -322,14 +366,15 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
     // output columns [nt*128 + half*64, +64): gate = weight row n, up = row up_row0 + n
     const int col0 = nt * 128 + half * 64;
     float h[64];
+    float ag[4], au[4];
+    seg_alpha4(c, p.nseg, col0, ag);
+    seg_alpha4(c, p.nseg, p.up_row0 + col0, au);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const float ag = seg_alpha(c, p.nseg, col0 + 16 * b);
-      const float au = seg_alpha(c, p.nseg, p.up_row0 + col0 + 16 * b);
 #pragma unroll
       for (int i = 16 * b; i < 16 * b + 16; ++i) {
-        const float g = ag * __uint_as_float(v[i >> 5][i & 31]);
-        const float u = au * __uint_as_float(v[2 + (i >> 5)][i & 31]);
+        const float g = ag[b] * __uint_as_float(v[i >> 5][i & 31]);
+        const float u = au[b] * __uint_as_float(v[2 + (i >> 5)][i & 31]);
         h[i] = silu_mul_f(g, u);
       }
     }
@@ -352,11 +397,12 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
     const int cg = col0 + 64 * hb;
     if (cg >= p.Nout) break;
     float y[64];
+    float a[4];
+    seg_alpha4(c, p.nseg, cg, a);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const float a = seg_alpha(c, p.nseg, cg + 16 * b);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) y[16 * b + i] = a * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
+      for (int i = 0; i < 16; ++i) y[16 * b + i] = a[b] * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
     }
     if (touches_gates(p, cg, 64)) gdn_gates<64>(p, row, cg, y);
     if (p.out_kind == OUT_NVFP4) {
@@ -379,6 +425,7 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
 __device__ __forceinline__ void store_partial(const Params &p, const uint32_t (&v)[4][32], int split, int row,
                                               int col0) {
   if (row >= p.M) return;
+  if (!NVFP4_DCHECK(split >= 0 && split < p.splits && col0 >= 0 && col0 % 16 == 0)) return;
   float *dst = p.partial + ((int64_t)split * p.M + row) * p.N + col0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -856,6 +903,53 @@ struct CtrlD {
 };
 static_assert(sizeof(CtrlD) <= PlanD::CTRL_BYTES, "control block too large");
 
+// Unsplit decode linear, epilogue applied in place of the FP32 partials (no reduction
+// kernel): output column n of every token row, y = alpha_seg(n) * acc, the GDN gate of
+// column n where it is one, stored as BF16 or FP32 (the launch takes this path only
+// for one split, epilogue none or GDN gates, and a BF16 / FP32 output).  The same
+// arithmetic as splitk_epilogue_kernel on a single split, element by element.
+__device__ __forceinline__ void decode_direct_epilogue(const Params &p, int n, const uint32_t (&v)[2][32]) {
+  float alpha = 0.0f;
+  for (int s = 0; s < p.nseg; ++s)
+    if (n >= p.seg[s].n_begin && n < p.seg[s].n_end)
+      alpha = __frcp_rn(__fmul_rn(__ldg(p.gs_a), __ldg(p.seg[s].gs_w)));
+  int gate = 0, hh = 0;  // 1: beta column (sigmoid), 2: alpha column (decay)
+  float la = 0.0f, db = 0.0f;
+  if (p.mode == MODE_GDN) {
+    if (n >= p.beta_begin && n < p.beta_begin + p.n_heads) {
+      gate = 1;
+      hh = n - p.beta_begin;
+    } else if (n >= p.alpha_begin && n < p.alpha_begin + p.n_heads) {
+      gate = 2;
+      hh = n - p.alpha_begin;
+      la = -__expf(__ldg(p.A_log + hh));
+      db = __ldg(p.dt_bias + hh);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && p.dn <= 32) break;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int m = 32 * h + i;
+      if (m >= p.M) break;
+      float y = alpha * __uint_as_float(v[h][i]);
+      if (gate == 1) {
+        y = sigmoid_f(y);
+        if (p.beta_out) p.beta_out[(int64_t)m * p.n_heads + hh] = y;
+      } else if (gate == 2) {
+        y = la * softplus_f(y + db);
+        if (p.g_out) p.g_out[(int64_t)m * p.n_heads + hh] = y;
+      }
+      if (!NVFP4_DCHECK(n >= 0 && n < p.Nout && m < p.M)) continue;
+      if (p.out_kind == OUT_BF16)
+        static_cast<__nv_bfloat16 *>(p.out)[(int64_t)m * p.ldo + n] = __float2bfloat16_rn(y);
+      else
+        static_cast<float *>(p.out)[(int64_t)m * p.ldo + n] = y;
+    }
+  }
+}
+
 // tmW: weight codes, boxes of 128 rows; tmX: token codes, boxes of p.dn rows.
 // p.sfb: the weight's scales, p.sfa: the tokens' (one 128-row group: p.M <= 64).
 __global__ void __launch_bounds__(DEC_THREADS, 1)
@@ -1004,7 +1098,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.acc_empty);
       const int n = nt * DEC_BM + 32 * q + lane;
-      if (n < p.N) {
+      if (n < p.N && p.partial == nullptr) {
+        decode_direct_epilogue(p, n, v);
+      } else if (n < p.N && NVFP4_DCHECK(split >= 0 && split < p.splits)) {
         float *dst = p.partial + (int64_t)split * p.M * p.N + n;
 #pragma unroll
         for (int m = 0; m < 32; ++m)
@@ -1071,13 +1167,16 @@ template <int W>
 __device__ __forceinline__ void store_w(const Params &p, int row, int col, const float (&y)[W]) {
   if constexpr (W == 16) {
     store16(p, row, col, y);
-  } else if (p.out_kind == OUT_BF16) {
-    const __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
-    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + col) =
-        make_uint2(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1));
-  } else if (p.out_kind == OUT_F32) {
-    *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (int64_t)row * p.ldo + col) =
-        make_float4(y[0], y[1], y[2], y[3]);
+  } else {
+    if (!NVFP4_DCHECK(row >= 0 && row < p.M && col >= 0 && col % W == 0 && col + W <= p.Nout)) return;
+    if (p.out_kind == OUT_BF16) {
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+      *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + col) =
+          make_uint2(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1));
+    } else if (p.out_kind == OUT_F32) {
+      *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (int64_t)row * p.ldo + col) =
+          make_float4(y[0], y[1], y[2], y[3]);
+    }
   }
 }
 
@@ -1085,6 +1184,7 @@ __device__ __forceinline__ void store_w(const Params &p, int row, int col, const
 // of store64_nvfp4.
 __device__ __forceinline__ void store16_nvfp4(const Params &p, const float *inv_out, int row, int col,
                                               const float (&y)[16], float gs_out) {
+  if (!NVFP4_DCHECK(row >= 0 && row < p.M && col >= 0 && col % 16 == 0 && col + 16 <= p.Nout)) return;
   float x[16];
   float amax = 0.0f;
 #pragma unroll

@@ -363,6 +363,10 @@ nvfp4_status_t prepare_linear(const nvfp4_operand_t *A, const float *gs_a, const
     p.out_scales = ep->out_scales;
     p.out_kb_atoms = Nout / 64;
   }
+  // 32-byte epilogue stores when every row of the output starts 32-byte aligned (an
+  // NVFP4 row is Nout / 2 bytes, a multiple of 32)
+  const int64_t row_bytes = out_kind == NVFP4_OUT_NVFP4 ? Nout / 2 : ldo * (out_kind == NVFP4_OUT_BF16 ? 2 : 4);
+  p.st32 = aligned(out, 32) && row_bytes % 32 == 0;
   return NVFP4_OK;
 }
 
@@ -400,8 +404,14 @@ nvfp4_status_t launch_splitk(gemm::Params p, const nvfp4_operand_t *A, const nvf
     const int64_t units = int64_t(p.n_tiles) * p.splits;
     if (units > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int grid = static_cast<int>(units < dev->sms ? units : dev->sms);
+    // One split, an element-wise epilogue and a BF16 / FP32 output: the kernel applies
+    // the epilogue itself (no partials, no reduction kernel).  SiLU*mul pairs columns of
+    // two tiles and an NVFP4 output needs 16 columns of a row; both keep the reduction.
+    const bool direct = p.splits == 1 && p.mode != MODE_SILU_MUL && p.out_kind != OUT_NVFP4;
+    if (direct) p.partial = nullptr;
     if (nvfp4_status_t e = launch_pdl(decode_kernel, dim3(grid), dim3(DEC_THREADS), PlanD::BYTES, st, 1, tmB, tmA, p))
       return e;
+    if (direct) return NVFP4_OK;
   } else {
     if (!make_codes_map(&tmA, A->codes, p.M, p.K) || !make_codes_map(&tmB, W->codes, p.N, p.K)) return NVFP4_ERR_CUDA;
     p.m_tiles = (p.M + BM - 1) / BM;

@@ -22,6 +22,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 }
 
 __device__ __forceinline__ void record_timeout() { atomicCAS(&g_device_status, 0, kStatusTimeout); }
+__device__ __forceinline__ void record_bad_index() { atomicCAS(&g_device_status, 0, kStatusBadIndex); }
+
+// Index invariant of a global store.  In the bounds-checking build (-DNVFP4_DEBUG, the
+// library libnvfp4_w4a4_debug.so) a violated invariant records NVFP4_ERR_DEVICE_INDEX
+// in the status word and the store is skipped; in the product build the check is
+// compiled out.  It stands in for a memory checker where none can run.
+#ifdef NVFP4_DEBUG
+#define NVFP4_DCHECK(cond) ((cond) ? true : (::nvfp4::record_bad_index(), false))
+#else
+#define NVFP4_DCHECK(cond) true
+#endif
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -124,6 +135,13 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, 
           smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// One 32-byte global store (sm_100 256-bit vector store); `dst` 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {

@@ -210,7 +210,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
     const int64_t dest = rt * kQTileRows + rho;
     const bool own = dest >= a.row_offset && dest < a.own_end;
     const int64_t col = ka * kQTileCols + 32 * h;
-    if (own && dest - a.row_offset < a.rows && col < a.cols) {
+    if (own && dest - a.row_offset < a.rows && col < a.cols &&
+        NVFP4_DCHECK(dest >= 0 && col % 32 == 0 && col / 2 + 8 <= a.code_ld)) {
       uint8_t *dst = a.codes + dest * a.code_ld + col / 2;
       if (col + 32 <= a.cols) {
         if (vec16) {
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
         uint4 *dst = reinterpret_cast<uint4 *>(a.scales + (rt * a.kb_atoms + ka) * 512);
         __stcg(dst + tid, reinterpret_cast<const uint4 *>(atom)[tid]);
       }
-    } else if (h == 0 && own) {
+    } else if (h == 0 && own && NVFP4_DCHECK(ka >= 0 && ka < a.kb_atoms)) {
       *reinterpret_cast<uint32_t *>(a.scales + scale_word_offset(dest, ka, a.kb_atoms)) = word;
     }
   }
@@ -263,6 +264,7 @@ __global__ void __launch_bounds__(kQSmallThreads) quantize_small_kernel(const ui
   if (idx >= (a.own_end - a.row_offset) * slots) return;
   const int64_t r = idx / slots, kb = idx - r * slots;
   const int64_t dest = a.row_offset + r;
+  if (!NVFP4_DCHECK(dest < a.own_end && kb < 4 * a.kb_atoms)) return;
   uint8_t *sc = a.scales + scale_word_offset(dest, kb / 4, a.kb_atoms) + (kb & 3);
   if (r >= a.rows || 16 * kb >= a.cols) {
     *sc = 0;

@@ -176,3 +176,16 @@ def test_layout_and_selftest_entry_points_reject_bad_arguments_without_launch(L)
     W2 = nv.Operand(1 << 22, 1 << 23, 512, 512)
     segs2 = (nv.Segment * 1)(nv.Segment(0, 512, 1 << 24))
     assert call(A, W2, segs2, 0) == 2                                     # two output tiles
+
+
+def test_debug_build_exports_the_same_boundary():
+    """The bounds-checking build (-DNVFP4_DEBUG) compiles and exports exactly the
+    declared entry points; it rejects bad arguments like the product build."""
+    path = nvbuild.build(debug=True)
+    out = os.popen(f"nm -D --defined-only {path}").read()
+    exported = {s for s in re.findall(r" T (\w+)", out) if s.startswith("nvfp4")}
+    assert exported == set(declared_symbols())
+    D = ctypes.CDLL(path)
+    fake = ctypes.c_void_p(1 << 20)
+    assert D.nvfp4_quantize(None, 4, 64, 64, fake, fake, fake, None) == 1
+    assert D.nvfp4_quantize(fake, 4, 24, 24, fake, fake, fake, None) == 2

@@ -79,6 +79,38 @@ def test_exact_narrow_last_n_tile(nv, M, N):
     assert nv.device_status() == 0
 
 
+@pytest.mark.parametrize("M", [100, 256])
+def test_outputs_only_16_byte_aligned(nv, M):
+    """The epilogue stores 32 bytes per lane when every output row starts 32-byte
+    aligned, else 16: a row stride of N + 8 BF16 / N + 4 FP32 elements, or a base 16
+    bytes past a 32-byte boundary, takes the 16-byte path and gives the same values
+    (and the NVFP4 output the same bytes)."""
+    import torch
+    K, N = 512, 384
+    xb = synth.student_t_activations(M, K, seed=90)
+    wb = synth.gaussian_weights(N, K, seed=91)
+    a = _quant_dev(nv, xb)
+    w = _quant_dev(nv, wb)
+    y16 = nv.linear(a, w, out_dtype="bf16")
+    y32 = nv.linear(a, w, out_dtype="f32")
+    b16 = torch.zeros((M, N + 8), dtype=torch.bfloat16, device="cuda")
+    b32 = torch.zeros((M, N + 4), dtype=torch.float32, device="cuda")
+    nv.linear(a, w, out_dtype="bf16", out=b16[:, :N])
+    nv.linear(a, w, out_dtype="f32", out=b32[:, :N])
+    flat16 = torch.zeros(M * N + 8, dtype=torch.bfloat16, device="cuda")
+    o16 = flat16[8:].view(M, N)  # base 16 bytes past a 32-byte boundary
+    nv.linear(a, w, out_dtype="bf16", out=o16)
+    gs_h = nv.global_scale(y16)
+    q_ref = nv.linear(a, w, out_dtype="nvfp4", gs_out=gs_h)
+    flat8 = torch.zeros(M * N // 2 + 16, dtype=torch.uint8, device="cuda")
+    q = nv.linear(a, w, out_dtype="nvfp4", gs_out=gs_h, out=flat8[16:].view(M, N // 2))
+    _sync()
+    assert torch.equal(b16[:, :N], y16) and torch.equal(o16, y16) and torch.equal(b32[:, :N], y32)
+    assert (b16[:, N:] == 0).all() and (b32[:, N:] == 0).all()
+    assert torch.equal(q.codes, q_ref.codes) and torch.equal(q.scales, q_ref.scales)
+    assert nv.device_status() == 0
+
+
 @pytest.mark.parametrize("M", [128, 256])
 def test_single_nonzero_probes(nv, M):
     """One non-zero code / scale at a time lands in exactly one output element.
