@@ -2,8 +2,8 @@
 same kernels with an index check before every GEMM and quantiser global store, which
 records NVFP4_ERR_DEVICE_INDEX and skips the store when it fails.  A child process
 runs a spread of entry points on it (quantiser at TMA and decode sizes, the 1-CTA and
-CTA-pair GEMMs with segments, SiLU*mul with NVFP4 requant, split-K and the unsplit
-decode epilogue with GDN gates); every output must equal the product build's bit for
+CTA-pair GEMMs with segments, SiLU*mul with NVFP4 requant at prefill and decode size,
+split-K and the unsplit decode epilogue with GDN gates); every output must equal the product build's bit for
 bit and the status word must stay clean."""
 import os
 import subprocess
@@ -43,6 +43,8 @@ def run():
     out["h16"], out["hq_codes"], out["hq_scales"] = h16, hq.codes, hq.scales
     a32 = nv.quantize(x[:32])
     out["splitk2"] = nv.linear_splitk(a32, w, segments=segs, out_dtype="bf16", split_k=2)
+    gq = nv.linear_splitk(a32, gu, segments=gsegs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=gs_h, split_k=1)
+    out["gu_dec_codes"], out["gu_dec_scales"] = gq.codes, gq.scales
     beta = torch.zeros((32, 16), dtype=torch.float32, device="cuda")
     g = torch.zeros((32, 16), dtype=torch.float32, device="cuda")
     gates = dict(beta_begin=432, alpha_begin=448, n_heads=16,

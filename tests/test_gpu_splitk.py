@@ -158,6 +158,46 @@ def test_silu_mul_requant_decode(nv, split_k):
     assert np.mean(gc == rc) > 0.995 and np.mean(gsf == rsf) > 0.995
 
 
+@pytest.mark.parametrize("M", [1, 20, 33, 64])
+def test_silu_mul_unsplit_decode(nv, M):
+    """One split at decode size: SiLU*mul (and the NVFP4 requant) over the gate and up
+    halves of the fused weight.  Token counts on both sides of the 32-row MMA width;
+    BF16 and FP32 against the oracle, the NVFP4 output (scale buffer pre-filled with
+    0xAB, so padding rows must be zeroed) equal to the standalone quantiser of the BF16
+    output and to the oracle's quantiser of it."""
+    import torch
+    K, Nh = 768, 384
+    ws = synth.segmented_weights([("gate", Nh), ("up", Nh)], K, seed=72, multipliers={"gate": 1, "up": 3})
+    xb = synth.student_t_activations(M, K, seed=73)
+    ca, sa, gsa = oracle_quant(xb)
+    oc, os_, oseg, n0 = [], [], [], 0
+    for _, wb in ws:
+        c, s, g = oracle_quant(wb)
+        oc.append(c), os_.append(s), oseg.append((n0, n0 + Nh, g))
+        n0 += Nh
+    y = oracle.linear(ca, sa, gsa, np.concatenate(oc), np.concatenate(os_), oseg)
+    h_ref = oracle.silu_mul(y[:, :Nh], y[:, Nh:])
+    w, dsegs = nv.quantize_fused([to_dev_bf16(wb) for _, wb in ws])
+    a = nv.quantize(to_dev_bf16(xb))
+    h16 = nv.linear_splitk(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="bf16", split_k=1)
+    h32 = nv.linear_splitk(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="f32", split_k=1)
+    _sync()
+    assert_gemm_close(h16, h_ref)
+    assert rel_fro(h32.cpu().numpy(), h_ref) <= 1e-3
+    assert torch.equal(h32.to(torch.bfloat16), h16)
+    gs_h = nv.global_scale(h16)
+    scales = torch.full((nv.scale_bytes(M, Nh),), 0xAB, dtype=torch.uint8, device="cuda")
+    hq = nv.linear_splitk(a, w, segments=dsegs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=gs_h,
+                          out_scales=scales, split_k=1)
+    hq2 = nv.quantize(h16, gs_h)
+    _sync()
+    assert torch.equal(hq.codes, hq2.codes) and torch.equal(hq.scales, hq2.scales)
+    gc, gsf = logical(hq)
+    kc, ks = oracle.quantize(h16.float().cpu().numpy(), np.float32(gs_h.item()))
+    assert np.array_equal(gc, kc) and np.array_equal(gsf, ks)
+    assert nv.device_status() == 0
+
+
 def test_bad_split_and_workspace_rejected(nv):
     import torch
     from nvfp4_w4a4_quantized_02_b200 import NVFP4Error
