@@ -626,10 +626,15 @@ class HybridSweep(Workload):
     themselves are not linears): fixed Student-t tensors of width 4096 / 6144.
     """
 
-    def __init__(self, nv, M=32768, seed=0):
+    def __init__(self, nv, M=32768, seed=0, layers=64):
         import torch
         self.nv, self.M = nv, M
-        self.name = f"hybrid_sweep_496_linears_m{M}"
+        self.n_layers = layers
+        self.n_gdn = sum(1 for li in range(layers) if li % 4 != 3)
+        self.n_attn = layers - self.n_gdn
+        self.n_linears = 5 * self.n_gdn + 4 * self.n_attn + 3 * layers
+        self.name = (f"hybrid_sweep_496_linears_m{M}" if layers == 64
+                     else f"hybrid_sweep_{self.n_linears}_linears_{layers}_layers_m{M}")
         H, I = 5120, 17408
         dev = "cuda"
         # activations per distinct input width, each with a static calibrated global scale
@@ -653,7 +658,7 @@ class HybridSweep(Workload):
         self.gates = _gdn_gate_tensors(torch, M, seed + 100)
         self.layers = []
         s = seed + 1000
-        for li in range(64):
+        for li in range(layers):
             L = {}
             if li % 4 == 3:
                 qkv = [_gpu_normal(6144, H, s, 0.02), _gpu_normal(1024, H, s + 1, 0.02),
@@ -678,31 +683,33 @@ class HybridSweep(Workload):
         self.gs_h = nv.global_scale(h16)
         del h16
         torch.cuda.synchronize()
-        per_tok = (48 * 2 * (12352 * H + H * 4096) + 16 * 2 * (8192 * H + H * 6144)
-                   + 64 * 2 * (2 * I * H + H * I))
+        ng, na, nl = self.n_gdn, self.n_attn, layers
+        per_tok = (ng * 2 * (12352 * H + H * 4096) + na * 2 * (8192 * H + H * 6144)
+                   + nl * 2 * (2 * I * H + H * I))
         self.flops = float(per_tok) * M
         self.f_gu = 2.0 * M * 2 * I * H
-        self.launches_per_step = 48 * 4 + 16 * 4 + 64 * 3
+        self.launches_per_step = ng * 4 + na * 4 + nl * 3
         self.packed_bytes = sum(t.codes.numel() + t.scales.numel()
                                 for L in self.layers for v in L.values()
                                 for t in ([v[0]] if isinstance(v, tuple) else [v]))
         self.l2_note = f"weights {self.packed_bytes / 2**30:.2f} GiB packed, streamed once per step (> L2)"
         self.dominant = ("gemm_gate_up", self.f_gu, "tensor",
                          "gemm2_kernel (CTA pair; MLP gate|up, SiLU*mul, NVFP4 requant epilogue)")
-        self.phases = {"quantize": ("GB/s", 2.5625 * M * (128 * H + 48 * 4096 + 16 * 6144)),
-                       "gemm_gdn_in": ("TFLOP/s", 48 * 2.0 * M * 12352 * H),
-                       "gemm_gdn_out": ("TFLOP/s", 48 * 2.0 * M * H * 4096),
-                       "gemm_attn_qkv": ("TFLOP/s", 16 * 2.0 * M * 8192 * H),
-                       "gemm_attn_o": ("TFLOP/s", 16 * 2.0 * M * H * 6144),
-                       "gemm_gate_up": ("TFLOP/s", 64 * self.f_gu),
-                       "gemm_down": ("TFLOP/s", 64 * 2.0 * M * H * I)}
+        self.phases = {"quantize": ("GB/s", 2.5625 * M * (2 * nl * H + ng * 4096 + na * 6144)),
+                       "gemm_gdn_in": ("TFLOP/s", ng * 2.0 * M * 12352 * H),
+                       "gemm_gdn_out": ("TFLOP/s", ng * 2.0 * M * H * 4096),
+                       "gemm_attn_qkv": ("TFLOP/s", na * 2.0 * M * 8192 * H),
+                       "gemm_attn_o": ("TFLOP/s", na * 2.0 * M * H * 6144),
+                       "gemm_gate_up": ("TFLOP/s", nl * self.f_gu),
+                       "gemm_down": ("TFLOP/s", nl * 2.0 * M * H * I)}
 
     def work(self):
         return self.flops
 
     def config(self):
-        return {"M": self.M, "layers": "48 GDN + 16 attention, 64 MLP", "linears": 496,
-                "gemm_launches_per_step": 256, "packed_weight_gib": round(self.packed_bytes / 2**30, 3),
+        return {"M": self.M, "layers": f"{self.n_gdn} GDN + {self.n_attn} attention, {self.n_layers} MLP",
+                "linears": self.n_linears, "gemm_launches_per_step": 2 * self.n_layers + 2 * self.n_layers,
+                "packed_weight_gib": round(self.packed_bytes / 2**30, 3),
                 "step": "per layer: quantise(input) -> fused NVFP4 GEMM(s) with the layer's epilogue"}
 
     def plan(self, x):
@@ -815,15 +822,24 @@ class DecodeSweep(HybridSweep):
     replayed as one CUDA graph (launch overhead would otherwise dominate)."""
     use_graph = True
 
-    def __init__(self, nv, M=32, seed=0):
+    def __init__(self, nv, M=32, seed=0, layers=64):
         import torch
-        super().__init__(nv, M=M, seed=seed)
-        self.name = f"decode_sweep_496_linears_m{M}"
+        super().__init__(nv, M=M, seed=seed, layers=layers)
+        self.name = (f"decode_sweep_496_linears_m{M}" if layers == 64
+                     else f"decode_sweep_{self.n_linears}_linears_{layers}_layers_m{M}")
         shapes = [(12352, 5120), (5120, 4096), (8192, 5120), (5120, 6144), (34816, 5120), (5120, 17408)]
         ws = max(nv.splitk_workspace_bytes(M, n, nv.splitk_default(M, n, k)) for n, k in shapes)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device="cuda")
         self.splits = {f"{n}x{k}": nv.splitk_default(M, n, k) for n, k in shapes}
-        self.launches_per_step = 48 * 4 + 16 * 4 + 64 * 3 + 256  # + one split-K epilogue launch per GEMM
+        ng, na, nl = self.n_gdn, self.n_attn, layers
+        # + one split-K epilogue launch per GEMM, except where one split lets the decode
+        # kernel apply the epilogue itself (element-wise epilogue, BF16 out: every GEMM
+        # of the step but the MLP gate|up with its NVFP4 output), or, above 64 rows, runs
+        # the plain GEMM
+        one = lambda key: int(self.splits[key] == 1)
+        direct = (ng * (one("12352x5120") + one("5120x4096")) + na * (one("8192x5120") + one("5120x6144"))
+                  + nl * one("5120x17408") + (nl * one("34816x5120") if M > 64 else 0))
+        self.launches_per_step = ng * 4 + na * 4 + nl * 3 + (2 * ng + 2 * na + 2 * nl) - direct
         H, I = 5120, 17408
         wb = lambda n, k: n * k * 0.5625  # packed codes + scales
 
@@ -833,13 +849,13 @@ class DecodeSweep(HybridSweep):
         self.dominant = ("gemm_gate_up", self.bytes_gu, "hbm",
                          f"nvfp4_linear_splitk (MLP gate|up, SiLU*mul, NVFP4 requant; "
                          f"split_k {self.splits['34816x5120']})")
-        self.phases = {"quantize": ("GB/s", 2.5625 * M * (128 * H + 48 * 4096 + 16 * 6144)),
-                       "gemm_gdn_in": ("GB/s", gemm_bytes(12352, H, 48)),
-                       "gemm_gdn_out": ("GB/s", gemm_bytes(H, 4096, 48)),
-                       "gemm_attn_qkv": ("GB/s", gemm_bytes(8192, H, 16)),
-                       "gemm_attn_o": ("GB/s", gemm_bytes(H, 6144, 16)),
-                       "gemm_gate_up": ("GB/s", 64 * self.bytes_gu),
-                       "gemm_down": ("GB/s", gemm_bytes(H, I, 64))}
+        self.phases = {"quantize": ("GB/s", 2.5625 * M * (2 * nl * H + ng * 4096 + na * 6144)),
+                       "gemm_gdn_in": ("GB/s", gemm_bytes(12352, H, ng)),
+                       "gemm_gdn_out": ("GB/s", gemm_bytes(H, 4096, ng)),
+                       "gemm_attn_qkv": ("GB/s", gemm_bytes(8192, H, na)),
+                       "gemm_attn_o": ("GB/s", gemm_bytes(H, 6144, na)),
+                       "gemm_gate_up": ("GB/s", nl * self.bytes_gu),
+                       "gemm_down": ("GB/s", gemm_bytes(H, I, nl))}
         self.l2_note = (f"weights {self.packed_bytes / 2**30:.2f} GiB packed, streamed from HBM once per step "
                         "(> L2)")
 
@@ -982,6 +998,10 @@ def make_workload(args, nv):
     kw = {}
     if args.M:
         kw["M"] = args.M
+    if args.layers:
+        if cls not in (HybridSweep, DecodeSweep):
+            raise SystemExit("--layers applies to the sweep and decode workloads")
+        kw["layers"] = args.layers
     return cls(nv, **kw)
 
 
@@ -1492,6 +1512,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mlp")
     ap.add_argument("--M", type=int, default=0, help="token rows (default: the workload's own)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="sweep / decode: build only the first L of the 64 layers (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="replay each step as one CUDA graph")
     ap.add_argument("--no-other-configs", action="store_true",
