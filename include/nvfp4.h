@@ -67,6 +67,17 @@ NVFP4_API const char *nvfp4_status_string(int status);
 NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t cols);
 
 /*
+ * nvfp4_amax - max|x| of a BF16 tensor, written as FP32 to *amax_out (device).  The
+ *   calibration step behind static global scales (blog section 罠①: every module keeps
+ *   the global scale it was calibrated with): run it over calibration inputs and
+ *   derive gs = 2688 / amax (the formula of nvfp4_global_scale) on the caller's side.
+ *   Exact (a maximum of BF16 magnitudes).  Same requirements and errors as
+ *   nvfp4_global_scale.
+ */
+NVFP4_API nvfp4_status_t nvfp4_amax(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *amax_out,
+                                    nvfp4_stream_t stream);
+
+/*
  * nvfp4_global_scale - per-tensor FP32 global scale from the tensor's amax.
  *   Computes gs = fl32(2688 / max|x|) over x [rows x cols] (row stride `ld`
  *   elements) and writes it to *gs_out (device).  max|x| == 0 gives gs = 1.

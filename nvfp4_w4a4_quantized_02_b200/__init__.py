@@ -13,7 +13,7 @@ from dataclasses import dataclass
 from typing import Optional, Sequence
 
 __all__ = [
-    "lib", "NVFP4Error", "scale_bytes", "global_scale", "quantize", "quantize_fused", "linear",
+    "lib", "NVFP4Error", "scale_bytes", "amax", "global_scale", "quantize", "quantize_fused", "linear",
     "linear_splitk", "linear_splitk_noalloc", "noalloc_default_splits", "splitk_default", "splitk_workspace_bytes",
     "NOALLOC_SCRATCH_BYTES", "fold_segments", "fp8_scale", "kv_cache_fp8", "gdn_recurrence",
     "device_status", "selftest_stalled_linear", "unswizzle_scales", "pack_weight", "NVFP4Tensor", "EPILOGUES", "OUT_KINDS",
@@ -59,7 +59,7 @@ SYMBOLS = ("nvfp4_status_string", "nvfp4_scale_bytes", "nvfp4_global_scale", "nv
            "nvfp4_quantize_rows", "nvfp4_linear", "nvfp4_linear_splitk", "nvfp4_splitk_workspace_bytes",
            "nvfp4_splitk_default", "nvfp4_linear_splitk_noalloc", "nvfp4_fold_segments",
            "nvfp4_fp8_scale", "nvfp4_kv_cache_fp8", "nvfp4_gdn_recurrence", "nvfp4_get_device_status",
-           "nvfp4_selftest_stalled_linear", "nvfp4_unswizzle_scales", "nvfp4_pack_weight")
+           "nvfp4_selftest_stalled_linear", "nvfp4_unswizzle_scales", "nvfp4_pack_weight", "nvfp4_amax")
 
 
 def lib():
@@ -76,6 +76,8 @@ def lib():
     L.nvfp4_status_string.argtypes = [ctypes.c_int]
     L.nvfp4_scale_bytes.restype = ctypes.c_size_t
     L.nvfp4_scale_bytes.argtypes = [_c_i64, _c_i64]
+    L.nvfp4_amax.restype = ctypes.c_int
+    L.nvfp4_amax.argtypes = [_c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp]
     L.nvfp4_global_scale.restype = ctypes.c_int
     L.nvfp4_global_scale.argtypes = [_c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp]
     L.nvfp4_quantize.restype = ctypes.c_int
@@ -159,6 +161,17 @@ class NVFP4Tensor:
     gs: "torch.Tensor"      # float32 [1]
     rows: int
     cols: int
+
+
+def amax(x, out=None, stream=None):
+    """max|x| of a 2-D BF16 CUDA tensor, as a float32 [1] device tensor (calibration)."""
+    import torch
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_cuda
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().nvfp4_amax(_c_vp(x.data_ptr()), x.shape[0], x.shape[1], x.stride(0), _c_vp(out.data_ptr()),
+                            _stream(stream)), "nvfp4_amax")
+    return out
 
 
 def global_scale(x, out=None, stream=None):

@@ -458,6 +458,24 @@ nvfp4_status_t noalloc_scratch(float **ptr) {
   return NVFP4_OK;
 }
 
+// max|x| of a BF16 matrix into *out (device FP32): zero it, then the amax kernel's
+// atomicMax over the bit patterns (non-negative floats order as unsigned integers).
+nvfp4_status_t launch_amax(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *out,
+                           const DeviceInfo *dev, cudaStream_t s) {
+  if (cudaMemsetAsync(out, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  AmaxArgs a;
+  a.x = static_cast<const uint16_t *>(x_bf16);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.amax_bits = reinterpret_cast<unsigned int *>(out);
+  const int64_t vecs = rows * (cols / 8);
+  const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
+  const int64_t cap = int64_t(dev->sms) * 4;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
+  return launch_pdl(amax_kernel, dim3(grid), dim3(kAmaxThreads), 0, s, 1, a);
+}
+
 }  // namespace
 
 extern "C" {
@@ -483,6 +501,17 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
   return static_cast<size_t>(rows_pad * kb_pad);
 }
 
+nvfp4_status_t nvfp4_amax(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *amax_out,
+                          nvfp4_stream_t stream) {
+  NvtxRange nvtx("nvfp4_amax");
+  if (!x_bf16 || !amax_out || rows < 1 || cols < 1 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0 || rows > kMaxDim || cols > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x_bf16, 16) || ld % 8 != 0 || !aligned(amax_out, 4)) return NVFP4_ERR_MISALIGNED;
+  DeviceInfo *dev = nullptr;
+  if (nvfp4_status_t st = current_device(&dev)) return st;
+  return launch_amax(x_bf16, rows, cols, ld, amax_out, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
 nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, float *gs_out,
                                   nvfp4_stream_t stream) {
   NvtxRange nvtx("nvfp4_global_scale");
@@ -492,18 +521,7 @@ nvfp4_status_t nvfp4_global_scale(const void *x_bf16, int64_t rows, int64_t cols
   DeviceInfo *dev = nullptr;
   if (nvfp4_status_t st = current_device(&dev)) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(gs_out, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
-  AmaxArgs a;
-  a.x = static_cast<const uint16_t *>(x_bf16);
-  a.rows = rows;
-  a.cols = cols;
-  a.ld = ld;
-  a.amax_bits = reinterpret_cast<unsigned int *>(gs_out);
-  const int64_t vecs = rows * (cols / 8);
-  const int64_t want = (vecs / 4 + kAmaxThreads - 1) / kAmaxThreads;
-  const int64_t cap = int64_t(dev->sms) * 4;
-  const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
-  if (nvfp4_status_t e = launch_pdl(amax_kernel, dim3(grid), dim3(kAmaxThreads), 0, s, 1, a)) return e;
+  if (nvfp4_status_t e = launch_amax(x_bf16, rows, cols, ld, gs_out, dev, s)) return e;
   return launch_pdl(global_scale_finalize_kernel, dim3(1), dim3(1), 0, s, 1, gs_out);
 }
 

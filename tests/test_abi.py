@@ -189,3 +189,14 @@ def test_debug_build_exports_the_same_boundary():
     fake = ctypes.c_void_p(1 << 20)
     assert D.nvfp4_quantize(None, 4, 64, 64, fake, fake, fake, None) == 1
     assert D.nvfp4_quantize(fake, 4, 24, 24, fake, fake, fake, None) == 2
+
+
+def test_amax_rejects_bad_arguments_without_launch(L):
+    vp = ctypes.c_void_p
+    f = vp(1 << 20)
+    assert L.nvfp4_amax(None, 4, 64, 64, f, None) == 1
+    assert L.nvfp4_amax(f, 4, 64, 64, None, None) == 1
+    assert L.nvfp4_amax(f, 4, 64, 60, f, None) == 1          # ld < cols
+    assert L.nvfp4_amax(f, 4, 72, 72, f, None) == 2          # cols % 16
+    assert L.nvfp4_amax(vp((1 << 20) + 2), 4, 64, 64, f, None) == 3
+    assert L.nvfp4_amax(f, 4, 64, 68, f, None) == 3          # ld % 8

@@ -137,3 +137,28 @@ def test_fused_pack_equals_separate_quantisation(nv):
     mask = np.ones(full.size, bool)
     mask[layout.scale_offset(r, j, 256).ravel()] = False
     assert np.all(full[mask] == 0)
+
+
+def test_amax_exact(nv):
+    """nvfp4_amax: max|x| exactly (a maximum of BF16 magnitudes), over a ragged matrix
+    read through a leading dimension wider than its columns, with the maximum on a
+    negative entry; an all-zero tensor gives 0, and global_scale is 2688 / amax."""
+    import torch
+    rows, cols, ld = 333, 496, 512
+    xb = synth.student_t_activations(rows, ld, seed=77)
+    x = synth.bf16_to_f32(xb)[:, :cols].copy()
+    r, c = 201, 417
+    x[r, c] = -4.0 * float(np.max(np.abs(x)))
+    # columns past `cols` hold a larger magnitude that the kernel must not read
+    bits = synth.f32_to_bf16_bits(np.pad(x, ((0, 0), (0, ld - cols)), constant_values=1.0e4))
+    dev = to_dev_bf16(bits)
+    view = dev[:, :cols]
+    got = nv.amax(view)
+    gs = nv.global_scale(view)
+    z = nv.amax(torch.zeros((4, 32), dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    ref = float(np.max(np.abs(synth.bf16_to_f32(bits)[:, :cols])))
+    assert float(got.item()) == ref
+    assert float(gs.item()) == float(oracle.global_scale(synth.bf16_to_f32(bits)[:, :cols]))
+    assert float(z.item()) == 0.0
+    assert nv.device_status() == 0
