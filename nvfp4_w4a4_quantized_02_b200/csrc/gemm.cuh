@@ -228,6 +228,11 @@ __device__ __forceinline__ void seg_alpha4(const Ctrl<STAGES> &c, int nseg, int 
 // logarithm's absolute error stays below 1e-6.
 __device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float silu_mul_f(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+// silu_mul_f of two elements: the same operations, the sum and the products packed.
+__device__ __forceinline__ float2 silu_mul_f2(float2 g, float2 u) {
+  const float2 d = add_f32x2(make_float2(1.0f, 1.0f), make_float2(__expf(-g.x), __expf(-g.y)));
+  return mul_f32x2(make_float2(__fdividef(g.x, d.x), __fdividef(g.y, d.y)), u);
+}
 __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))); }
 
 // Store 16 consecutive output values of one row.
@@ -279,9 +284,11 @@ __device__ __forceinline__ void store64_nvfp4(const Params &p, const float *inv_
     float x[16];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      x[i] = __bfloat162float(__float2bfloat16_rn(y[16 * b + i]));
-      amax = fmaxf(amax, fabsf(x[i]));
+    for (int i = 0; i < 16; i += 2) {  // round to BF16 two at a time (RNE, as one by one)
+      const __nv_bfloat162 hb = __floats2bfloat162_rn(y[16 * b + i], y[16 * b + i + 1]);
+      x[i] = __low2float(hb);
+      x[i + 1] = __high2float(hb);
+      amax = fmaxf(amax, fmaxf(fabsf(x[i]), fabsf(x[i + 1])));
     }
     const uint32_t sf = block_scale_byte(amax, gs_out);
     const float inv = inv_out[sf & 127];
@@ -372,10 +379,15 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
 #pragma unroll
-      for (int i = 16 * b; i < 16 * b + 16; ++i) {
-        const float g = ag[b] * __uint_as_float(v[i >> 5][i & 31]);
-        const float u = au[b] * __uint_as_float(v[2 + (i >> 5)][i & 31]);
-        h[i] = silu_mul_f(g, u);
+      for (int i = 16 * b; i < 16 * b + 16; i += 2) {
+        const float2 g = mul_f32x2(make_float2(ag[b], ag[b]), make_float2(__uint_as_float(v[i >> 5][i & 31]),
+                                                                          __uint_as_float(v[i >> 5][(i & 31) + 1])));
+        const float2 u = mul_f32x2(make_float2(au[b], au[b]),
+                                   make_float2(__uint_as_float(v[2 + (i >> 5)][i & 31]),
+                                               __uint_as_float(v[2 + (i >> 5)][(i & 31) + 1])));
+        const float2 hh = silu_mul_f2(g, u);
+        h[i] = hh.x;
+        h[i + 1] = hh.y;
       }
     }
     if (p.out_kind == OUT_NVFP4) {
@@ -402,7 +414,12 @@ __device__ __forceinline__ void epilogue_row(const Params &p, const Ctrl<STAGES>
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) y[16 * b + i] = a[b] * __uint_as_float(v[2 * hb + (b >> 1)][(b & 1) * 16 + i]);
+      for (int i = 0; i < 16; i += 2) {
+        const uint32_t *src = &v[2 * hb + (b >> 1)][(b & 1) * 16 + i];
+        const float2 r = mul_f32x2(make_float2(a[b], a[b]), make_float2(__uint_as_float(src[0]), __uint_as_float(src[1])));
+        y[16 * b + i] = r.x;
+        y[16 * b + i + 1] = r.y;
+      }
     }
     if (touches_gates(p, cg, 64)) gdn_gates<64>(p, row, cg, y);
     if (p.out_kind == OUT_NVFP4) {

@@ -314,6 +314,32 @@ __device__ __forceinline__ void tc_commit_cg2(uint64_t *bar) {
                : "memory");
 }
 
+// ------------------------------------------------------- packed FP32 (sm_100)
+// Two IEEE round-to-nearest products / sums in one instruction: the same results as
+// two scalar __fmul_rn / __fadd_rn, half the issue slots.
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "mul.rn.f32x2 z, x, y;\n\t"
+      "mov.b64 {%0, %1}, z;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "add.rn.f32x2 z, x, y;\n\t"
+      "mov.b64 {%0, %1}, z;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 // -------------------------------------------------------------- conversions
 // Round to E4M3 (nearest even, saturate to +-448): hi -> byte 1, lo -> byte 0.
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float hi, float lo) {

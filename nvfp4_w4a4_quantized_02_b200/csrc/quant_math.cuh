@@ -25,11 +25,16 @@ __device__ __forceinline__ uint32_t block_scale(float amax, float gs, float &inv
   return sf;
 }
 
-// Eight values -> eight E2M1 codes (element i in nibble i).
+// Eight values -> eight E2M1 codes (element i in nibble i).  The products x * inv are
+// IEEE round-to-nearest, two per packed instruction.
 __device__ __forceinline__ uint32_t encode8(const float *x, float inv) {
   float v[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[i], inv);
+  for (int i = 0; i < 8; i += 2) {
+    const float2 r = mul_f32x2(make_float2(x[i], x[i + 1]), make_float2(inv, inv));
+    v[i] = r.x;
+    v[i + 1] = r.y;
+  }
   return cvt_e2m1x8(v);
 }
 
