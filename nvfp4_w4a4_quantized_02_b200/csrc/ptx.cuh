@@ -65,20 +65,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test: has the phase with parity `parity` completed?  (Never suspends
-// the thread, so its latency can overlap independent instructions issued after it.)
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase with parity `parity` to complete.  Gives up after kLimit
 // polls (kMaxWaitIters unless a self-test instantiation asks for fewer), records a
 // timeout in the status word and returns false.
