@@ -8,7 +8,10 @@
 // section 機構② (GDN gates beta = sigmoid(b), g = -exp(A_log) * softplus(a + dt_bias)).
 //
 // Two kernels share the tile shape per CTA (128 output rows x 256 output columns,
-// K staged 256 FP4 elements = 128 bytes per row at a time) and the epilogue:
+// K staged 256 FP4 elements = 128 bytes per row at a time) and the epilogue; a last
+// N-tile narrower than 256 runs an MMA of its width rounded up to 32.  A third,
+// decode_kernel (further down), serves up to 64 token rows with the weight as the
+// MMA's 128-row side; splitk_epilogue_kernel reduces split-K partial sums.
 //
 // gemm_kernel (1 CTA per tile, used when M <= 128): tcgen05.mma.cta_group::1,
 //   M = 128, N = 256; the CTA loads both 128-row halves of the B tile.
@@ -31,7 +34,11 @@
 //               per-stage loop: 2.47 -> 2.27 ms on the MLP block's gate|up GEMM.)
 //   warps 2..9  epilogue: tcgen05.ld the 128 x 256 FP32 accumulator (each warp a
 //               32-lane quadrant x 128 columns) into registers, hand TMEM back to the
-//               MMA warp at once, then scale / activate / store from registers.
+//               MMA warp at once, then scale / activate / store from registers.  Its
+//               warps share the sub-partitions (and their issue slots) with the
+//               producer, copier and MMA threads, so its instruction count shows in
+//               the mainloop: FP32 products and sums run two per packed instruction,
+//               and a lane stores 32 bytes at once where the output rows allow it.
 //   warps 10,11 scale copiers: per stage, 12 tcgen05.cp of the A and B scale atoms
 //               (6 per warp) into that stage's TMEM scale columns, then
 //               tcgen05.commit to the MMA issuer.  Issued from their own threads, the
