@@ -60,7 +60,8 @@ def test_exact_power_of_two_scales_pin_scale_layout(nv):
     assert np.array_equal(got, ref), f"{np.sum(got != ref)} mismatches"
 
 
-@pytest.mark.parametrize("M,N", [(100, 80), (256, 16), (256, 48), (256, 336), (300, 464), (512, 272), (128, 208)])
+@pytest.mark.parametrize("M,N", [(100, 80), (256, 16), (256, 48), (256, 336), (300, 464), (512, 272), (128, 208),
+                                 (257, 272), (511, 48)])
 def test_exact_narrow_last_n_tile(nv, M, N):
     """The last N-tile narrower than 256 runs an MMA of N = its width rounded up to 32;
     in the CTA pair the second CTA then holds B rows [N/2, N) of the tile.  Integer codes
@@ -76,6 +77,36 @@ def test_exact_narrow_last_n_tile(nv, M, N):
     _sync()
     got = out.cpu().numpy().astype(np.float64)
     assert np.array_equal(got, ref), f"{np.sum(got != ref)} mismatches"
+    assert nv.device_status() == 0
+
+
+def test_repeat_launches_bit_identical(nv):
+    """Race check: the CTA-pair kernel (SiLU*mul + NVFP4 requant, and BF16 out), the
+    1-CTA kernel and the decode-size split-K path, each launched four times back to back
+    on the same inputs, write the same bytes every time.  A stage or scale set reused
+    before its consumers finished, or an accumulator read before its MMAs completed,
+    would make launches differ."""
+    import torch
+    K = 2048
+    xb = synth.student_t_activations(1024, K, seed=95)
+    gu, gsegs = nv.quantize_fused([to_dev_bf16(synth.gaussian_weights(2048, K, seed=96)),
+                                   to_dev_bf16(synth.gaussian_weights(2048, K, seed=97, std=0.04))])
+    a = _quant_dev(nv, xb)
+    a100 = _quant_dev(nv, xb[:100])
+    a32 = _quant_dev(nv, xb[:32])
+    h16 = nv.linear(a, gu, segments=gsegs, epilogue="silu_mul", out_dtype="bf16")
+    gs_h = nv.global_scale(h16)
+    runs = {"pair_nvfp4": [], "pair_bf16": [], "one_cta": [], "decode": []}
+    for _ in range(4):
+        q = nv.linear(a, gu, segments=gsegs, epilogue="silu_mul", out_dtype="nvfp4", gs_out=gs_h)
+        runs["pair_nvfp4"].append(torch.cat([q.codes.flatten(), q.scales]))
+        runs["pair_bf16"].append(nv.linear(a, gu, segments=gsegs, out_dtype="bf16"))
+        runs["one_cta"].append(nv.linear(a100, gu, segments=gsegs, out_dtype="f32"))
+        runs["decode"].append(nv.linear_splitk(a32, gu, segments=gsegs, out_dtype="bf16", split_k=2))
+    _sync()
+    for k, outs in runs.items():
+        for o in outs[1:]:
+            assert torch.equal(o, outs[0]), k
     assert nv.device_status() == 0
 
 
