@@ -51,6 +51,11 @@ METRIC = "NVFP4 W4A4 linear TFLOPS & % of B200 dense FP4 peak; quantise GB/s vs 
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 NOMINAL_FP4_TFLOPS = 9000.0  # datasheet dense NVFP4 tensor peak of one B200
 NOMINAL_HBM_GBS = 8000.0     # datasheet HBM3e bandwidth of one B200 (~8 TB/s)
+# TMA operand bytes one K stage of a 256 x 256 CTA-pair tile brings from L2 into the pair's
+# shared memory: per CTA 128 A rows and 128 B rows of 128 bytes (256 FP4), A's scale atoms
+# (2 KB) and both halves of B's (4 KB).  At full occupancy the pair GEMM is bound by this
+# stream (~12 TB/s measured by timing it on fewer clusters).
+PAIR_STAGE_L2_BYTES = 2 * (128 * 128 + 128 * 128 + 2048 + 4096)
 SUSTAINED_REGION_MS = 1000.0  # timed regions at least this long use the sustained GEMM peak
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP32_LANES_PER_SM = 128     # FP32 FMA lanes per SM (4 sub-partitions x 32)
@@ -151,6 +156,12 @@ def sources_hash(files):
         with open(os.path.join(d, fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
+
+
+def pair_gemm_l2_bytes(M, N, K):
+    """L2 -> SM operand bytes of one CTA-pair GEMM launch (M > 128, N and K multiples of
+    256): tiles x K stages x PAIR_STAGE_L2_BYTES."""
+    return -(-M // 256) * (N // 256) * (K // 256) * PAIR_STAGE_L2_BYTES
 
 
 def load_traffic(key):
@@ -396,6 +407,9 @@ class MLPBlock(Workload):
                          "gemm2_kernel (CTA pair; gate|up, SiLU*mul, NVFP4 requant epilogue)")
         self.phases = {"global_scale": ("GB/s", 2.0 * M * H), "quantize": ("GB/s", 2.5625 * M * H),
                        "gemm_gate_up": ("TFLOP/s", self.f_gu), "gemm_down": ("TFLOP/s", self.f_d)}
+        if M > 128:  # CTA-pair kernels: their L2 -> SM operand stream
+            self.l2_stream = {"gemm_gate_up": pair_gemm_l2_bytes(M, 2 * I, H),
+                              "gemm_down": pair_gemm_l2_bytes(M, H, I)}
 
     def work(self):
         return self.f_gu + self.f_d
@@ -1130,6 +1144,8 @@ def run_ours(args, ws, rank):
             d["TFLOP/s"] = round(amount / ms / 1e9, 1)
             d["frac_fp4_peak"] = round(d["TFLOP/s"] / fp4_peak, 4)
             d["frac_fp4_nominal"] = round(d["TFLOP/s"] / NOMINAL_FP4_TFLOPS, 4)
+        if key in getattr(wl, "l2_stream", {}):
+            d["l2_to_sm_TB/s"] = round(wl.l2_stream[key] / (ms / per_phase[key]["launches"]) / 1e9, 2)
         kernels[key] = d
 
     key, per_launch, bound, label = wl.dominant
@@ -1166,6 +1182,12 @@ def run_ours(args, ws, rank):
             extra_fracs["frac_nominal_at_median_clock"] = round(achieved / fp4_at_clock, 4)
     if sm_mhz:
         extra_fracs["sm_mhz_median"] = sm_mhz
+    if key in getattr(wl, "l2_stream", {}):
+        extra_fracs["l2_to_sm"] = {
+            "TB/s": round(wl.l2_stream[key] / avg_ms / 1e9, 2), "bytes_per_launch": wl.l2_stream[key],
+            "note": "TMA operand bytes from L2 (76 KB per 256x256x256 pair-tile stage) / launch time; at full "
+                    "occupancy the pair GEMM runs at this stream's ~12 TB/s limit (same rate for gate|up and down; "
+                    "per-tile time falls to the MMA stream's on fewer clusters)"}
     roof = {"kernel": label, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), **extra_fracs, "traffic": load_traffic(f"{key}@{wl.name}"),
             "avg_launch_ms": round(avg_ms, 5), "work_per_launch": per_launch, "peak_note": note,
