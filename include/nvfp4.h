@@ -412,8 +412,8 @@ NVFP4_API nvfp4_status_t nvfp4_get_device_status(int *code);
  * producer skips stage `stall_stage` (counted from 0 over the K tiles), so the scale
  * copiers and the MMA issuer wait on a barrier phase that never completes, and the
  * epilogue waits on an accumulator that is never committed.  In this instantiation
- * every wait gives up after a short limit (4096 polls instead of the product's
- * 2^22): each role records NVFP4_ERR_DEVICE_TIMEOUT in the device status word, waits
+ * every wait gives up after a short limit (1 ms instead of the product's 0.5 s):
+ * each role records NVFP4_ERR_DEVICE_TIMEOUT in the device status word, waits
  * for the work it already issued, TMEM is freed and the kernel returns.  The output
  * is left partly written and is meaningless.  The context stays usable: read and
  * clear the status with nvfp4_get_device_status, after which the other entry points

@@ -501,7 +501,7 @@ __device__ __forceinline__ void cp_scale_atom(uint32_t taddr, uint32_t saddr) {
   }
 }
 
-template <int STAGES, bool kPair, uint32_t kWait = kMaxWaitIters>
+template <int STAGES, bool kPair, uint64_t kWait = kMaxWaitNs>
 __device__ __forceinline__ void copy_scales(Ctrl<STAGES> &c, uint32_t tmem, const uint8_t *sSFA,
                                             const uint8_t *sSFB, int total, int part) {
   int stage = 0;
@@ -561,7 +561,7 @@ __device__ __forceinline__ void init_barriers(Ctrl<STAGES> &c, uint32_t acc_empt
 // fetching instructions.
 // kStallTest: the failure-detection self-test.  The producer skips stage
 // p.stall_stage (no expected bytes, no loads), so the consumers of that stage wait for
-// a phase that never completes; every wait is capped at kTestWaitIters polls.  Each
+// a phase that never completes; every wait gives up after kTestWaitNs (1 ms).  Each
 // role then records NVFP4_ERR_DEVICE_TIMEOUT, waits for the work it already issued
 // and leaves; TMEM is freed and the kernel returns.
 template <bool kPartial, bool kStallTest = false>
@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const __grid_constant__ Params p) {
   using P = Plan1;
   constexpr int STAGES = P::STAGES;
-  constexpr uint32_t kWait = kStallTest ? kTestWaitIters : kMaxWaitIters;
+  constexpr uint64_t kWait = kStallTest ? kTestWaitNs : kMaxWaitNs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl<STAGES> &c = *reinterpret_cast<Ctrl<STAGES> *>(smem);

@@ -1,9 +1,9 @@
 """Failure detection on the GPU without a fault: every mbarrier wait in the library's
-kernels has an iteration limit, after which the kernel records NVFP4_ERR_DEVICE_TIMEOUT
+kernels has a time limit (0.5 s, read from the GPU's global timer), after which the kernel records NVFP4_ERR_DEVICE_TIMEOUT
 in the device status word, waits for its own work in flight, frees its TMEM and
 returns.  nvfp4_selftest_stalled_linear makes such a wait run out on purpose: the
 producer of the 1-CTA GEMM never loads one pipeline stage, and that instantiation's
-waits give up after 4096 polls.  The test checks the status read-back, that the read
+waits give up after 1 ms.  The test checks the status read-back, that the read
 clears it, and that the context then runs a normal linear to parity."""
 import numpy as np
 import pytest
