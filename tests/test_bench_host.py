@@ -66,3 +66,19 @@ def test_reference_arm_only_rank0_prints():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "linear_m128_n1024_k1024"
+
+
+def test_pair_gemm_l2_stream_bytes():
+    """The L2 -> SM operand bytes the bench reports for the CTA-pair GEMM: per 256 x 256
+    tile and 256-wide K stage, each CTA brings 128 A rows and 128 B rows of 128 bytes, A's
+    four 512-byte scale atoms and both 128-row halves of B's (eight atoms)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    per_cta = 128 * 128 + 128 * 128 + 4 * 512 + 8 * 512
+    assert bench.PAIR_STAGE_L2_BYTES == 2 * per_cta == 77824
+    # MLP gate|up at 32768 tokens: 128 x 136 pair tiles, 20 K stages
+    assert bench.pair_gemm_l2_bytes(32768, 34816, 5120) == 128 * 136 * 20 * 77824
+    # down projection: 128 x 20 tiles, 68 K stages
+    assert bench.pair_gemm_l2_bytes(32768, 5120, 17408) == 128 * 20 * 68 * 77824
+    # a ragged last M tile still loads a whole pair tile
+    assert bench.pair_gemm_l2_bytes(300, 256, 256) == 2 * 1 * 1 * 77824
