@@ -92,7 +92,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 // Wait for the phase with parity `parity` to complete.  Gives up kLimitNs after the
 // first unsuccessful poll (kMaxWaitNs unless a self-test instantiation asks for less),
 // records a timeout in the status word and returns false.  The limit is a time, not a
-// poll count, so it holds whatever the suspension between polls.
+// poll count, so it holds whatever the suspension between polls.  Time the kernel
+// spends preempted or slowed by an instrumenting tool counts too; a single wait of the
+// library's pipelines normally lasts microseconds (one stage, or one tile's main loop),
+// so 0.5 s leaves a margin of several orders of magnitude.
 template <uint64_t kLimitNs = kMaxWaitNs, bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   auto poll = [&] { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
