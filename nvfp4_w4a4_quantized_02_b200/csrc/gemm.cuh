@@ -47,7 +47,8 @@
 //               (measured on the MLP block's gate|up GEMM, 1-CTA kernel: 3.26 ms in
 //               line, 2.76 ms with one copier; CTA-pair kernel: 2.55 ms with one
 //               copier, 2.50 ms with two).
-// Output tiles are visited in groups of 16 M-tiles so that concurrently running
+// Output tiles are visited in groups of M-tiles (16, or 32 for a wide weight whose
+// group of A rows fits a quarter of L2; chosen by the host) so that concurrently running
 // CTAs share A and W tiles in L2.
 #pragma once
 
@@ -69,7 +70,7 @@ constexpr int NUM_EPI_WARPS = 8;
 constexpr int COPY_WARP = 2 + NUM_EPI_WARPS;  // first of the scale-copy warps
 constexpr int NUM_COPY_WARPS = 2;  // copy_scales splits a stage's 12 atoms in two halves
 constexpr int NUM_THREADS = 32 * (COPY_WARP + NUM_COPY_WARPS);
-constexpr int GROUP_M = 16;
+constexpr int GROUP_M = 16;        // M-tiles per raster group (Params::group_m), the default
 
 // TMEM columns (allocation of 512 = the whole TMEM of the SM): the 256-column FP32
 // accumulator, then one set of scale columns per shared-memory stage, so that the
@@ -142,6 +143,10 @@ struct Params {
   int stall_stage;
   // the output's base and row stride are 32-byte aligned: stores of 32 bytes per lane
   int st32;
+  // output tiles are visited in groups of group_m M-tiles (every N-tile of the group's
+  // rows before the next group), so that concurrently running CTAs share A and W tiles
+  // in L2; chosen by the host
+  int group_m;
 };
 
 template <int STAGES>
@@ -168,11 +173,11 @@ __host__ __device__ constexpr uint32_t make_idesc(int m, int n) {
 }
 
 __device__ __forceinline__ void tile_coords(const Params &p, int tile, int &mt, int &nt) {
-  const int per_group = GROUP_M * p.n_tiles;
+  const int per_group = p.group_m * p.n_tiles;
   const int g = tile / per_group;
   const int idx = tile - g * per_group;
-  const int gm = min(GROUP_M, p.m_tiles - g * GROUP_M);
-  mt = g * GROUP_M + idx % gm;
+  const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
+  mt = g * p.group_m + idx % gm;
   nt = idx / gm;
 }
 

@@ -367,6 +367,7 @@ nvfp4_status_t prepare_linear(const nvfp4_operand_t *A, const float *gs_a, const
   // NVFP4 row is Nout / 2 bytes, a multiple of 32)
   const int64_t row_bytes = out_kind == NVFP4_OUT_NVFP4 ? Nout / 2 : ldo * (out_kind == NVFP4_OUT_BF16 ? 2 : 4);
   p.st32 = aligned(out, 32) && row_bytes % 32 == 0;
+  p.group_m = GROUP_M;
   return NVFP4_OK;
 }
 
@@ -596,6 +597,12 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
     const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
     return launch_pdl(gemm_kernel<false>, dim3(grid), dim3(NUM_THREADS), Plan1::BYTES, st, 1, tmA, tmB, p);
   }
+  // A wide weight (64 N-tiles or more) is streamed from DRAM once per raster group:
+  // groups of 32 M-tiles halve those re-reads while the group's A rows (codes and
+  // scales) stay within a quarter of L2.  MLP gate|up at 32768 tokens: DRAM reads
+  // 895 -> 496 MB per launch, 1.6 % faster; a longer K (the down projection) keeps 16.
+  if (p.n_tiles >= 64 && int64_t(2 * GROUP_M) * (2 * BM) * (K / 2) * 9 / 8 <= (int64_t(32) << 20))
+    p.group_m = 2 * GROUP_M;
   const int64_t clusters = tiles < dev->gemm2_clusters ? tiles : dev->gemm2_clusters;
   return launch_pdl(gemm2_kernel, dim3(static_cast<unsigned>(2 * clusters)), dim3(NUM_THREADS), Plan2::BYTES, st, 2, tmA,
                     tmB, tmSFA, tmSFB, p);
