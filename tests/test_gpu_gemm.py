@@ -168,6 +168,26 @@ def test_single_nonzero_probes(nv, M):
 
 
 # ------------------------------------------------------- realistic parity
+def test_raster_groups_of_32_with_a_ragged_group(nv):
+    """A wide weight (64 N-tiles or more) whose group of A rows fits a quarter of L2 is
+    rastered in groups of 32 pair M-tiles; 33 M-tiles leave a last group of one.  Exact
+    integer case (all scales 1, gs 1: FP32 accumulation is exact).  One row in every
+    256-row pair tile, plus rows at tile and group boundaries, are compared with the
+    oracle over all columns, so every (M-tile, N-tile) pair of the launch is checked."""
+    rng = np.random.default_rng(7)
+    M, N, K = 33 * 256, 64 * 256, 256
+    ca = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    cw = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sa = np.full((M, K // 16), 0x38, np.uint8)
+    sw = np.full((N, K // 16), 0x38, np.uint8)
+    rows = sorted({256 * t + (37 * t) % 256 for t in range(33)} | {0, 127, 128, 255, 256, 8191, 8192, M - 1})
+    ref = oracle.linear(ca[rows], sa[rows], 1.0, cw, sw, [(0, N, 1.0)])
+    out = nv.linear(make_operand(ca, sa, 1.0), make_operand(cw, sw, 1.0), out_dtype="f32")
+    _sync()
+    got = out[rows].cpu().numpy().astype(np.float64)
+    assert np.array_equal(got, ref), f"{np.sum(got != ref)} mismatches"
+
+
 def _quant_dev(nv, bits, gs=None):
     x = to_dev_bf16(bits)
     return nv.quantize(x, None if gs is None else to_dev_f32([gs]))
