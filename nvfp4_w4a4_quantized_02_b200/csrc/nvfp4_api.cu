@@ -599,8 +599,9 @@ nvfp4_status_t nvfp4_linear(const nvfp4_operand_t *A, const float *gs_a, const n
   }
   // A wide weight (64 N-tiles or more) is streamed from DRAM once per raster group:
   // groups of 32 M-tiles halve those re-reads while the group's A rows (codes and
-  // scales) stay within 32 MB, a quarter of the B200's L2.  MLP gate|up at 32768 tokens: DRAM reads
-  // 895 -> 496 MB per launch, 1.6 % faster; a longer K (the down projection) keeps 16.
+  // scales) stay within 32 MB, a quarter of the B200's L2.  MLP gate|up at 32768
+  // tokens: DRAM reads 895 -> 496 MB per launch, 1.6 % faster; a longer K (the down
+  // projection) keeps 16.
   if (p.n_tiles >= 64 && int64_t(2 * GROUP_M) * (2 * BM) * (K / 2) * 9 / 8 <= (int64_t(32) << 20))
     p.group_m = 2 * GROUP_M;
   const int64_t clusters = tiles < dev->gemm2_clusters ? tiles : dev->gemm2_clusters;
